@@ -1,0 +1,203 @@
+"""Pins for the oracle's retention rule and slot-pool simulator (CPU only).
+
+What pins what:
+  * hand-derived traces (tests/golden/delayed_eviction_traces.txt) fix the
+    window bound and the slot-reuse order;
+  * the closed form n_s = (s+1) - #{j <= s-w : alpha_j = 1} and the dense
+    invariant (slots [0, n) occupied, ceil(n/16) pages) hold for random runs;
+  * brute force over every alpha pattern of length <= 12 compares the
+    simulator (ring-free lookup, slot reuse) with the visibility definition;
+  * a hand-derived free-stack trace (tests/golden/page_pops.txt) fixes the
+    page-pop and reset order.
+"""
+import os
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _parse_traces():
+    traces, cur = [], None
+    for line in open(os.path.join(GOLD, "delayed_eviction_traces.txt")):
+        line = line.split("#", 1)[0].strip()
+        if not line:
+            continue
+        key, _, rest = line.partition(" ")
+        if key == "trace":
+            cur = {"name": rest, "visible": {}}
+            traces.append(cur)
+        elif key == "window":
+            cur["w"] = int(rest)
+        elif key == "alpha":
+            cur["alpha"] = [int(x) for x in rest.split()]
+        elif key == "visible":
+            s, _, pos = rest.partition(":")
+            cur["visible"][int(s)] = [int(x) for x in pos.split()]
+        elif key == "slots":
+            cur["slots"] = [int(x) for x in rest.split()]
+        elif key == "final":
+            cur["final"] = [int(x) for x in rest.split()]
+    return traces
+
+
+TRACES = _parse_traces()
+
+
+@pytest.mark.parametrize("tr", TRACES, ids=[t["name"] for t in TRACES])
+def test_golden_visible_sets(tr):
+    a, w = tr["alpha"], tr["w"]
+    assert len(tr["visible"]) == len(a)
+    for s, expect in tr["visible"].items():
+        assert oracle.visible_positions(a, s, w) == expect
+        got_c = [j for j in range(s + 1) if oracle.lib().dmso_visible(s, j, a[j], w)]
+        assert got_c == expect
+        assert oracle.retained_count_closed_form(a, s, w) == len(expect)
+
+
+@pytest.mark.parametrize("tr", TRACES, ids=[t["name"] for t in TRACES])
+def test_golden_slots(tr):
+    a, w = tr["alpha"], tr["w"]
+    sim = oracle.Sim(1, 1, w, max_pages=4, max_pages_per_stream=4)
+    logical = []
+    for s, bit in enumerate(a):
+        rc, phys = sim.append([0], [1], np.array([[bit]], dtype=np.uint8), want_slots=True)
+        assert rc == 0
+        snap = sim.snapshot()
+        page = int(phys[0, 0]) // 16
+        logical_page = list(snap["page_table"][0]).index(page)
+        logical.append(logical_page * 16 + int(phys[0, 0]) % 16)
+        assert sorted(sim.retained(0).tolist()) == tr["visible"][s]
+    assert logical == tr["slots"]
+    assert sim.retained(0).tolist() == tr["final"]
+
+
+def test_visible_rule_edges():
+    vis = oracle.lib().dmso_visible
+    assert vis(5, 6, 0, 3) == 0          # future position
+    assert vis(5, -1, 0, 3) == 0
+    assert vis(5, 5, 1, 1) == 1          # own token always visible (w >= 1)
+    assert vis(5, 4, 1, 1) == 0
+    assert vis(5, 3, 1, 3) == 1          # age 2 < 3
+    assert vis(5, 2, 1, 3) == 0          # age 3 == w -> gone
+    assert vis(10**6, 0, 0, 1) == 1      # kept tokens stay forever
+
+
+def test_c_and_python_rule_agree():
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        T = int(rng.integers(1, 60))
+        w = int(rng.integers(1, 70))
+        a = rng.integers(0, 2, T).tolist()
+        s = T - 1
+        py = oracle.visible_positions(a, s, w)
+        c = [j for j in range(T) if oracle.lib().dmso_visible(s, j, a[j], w)]
+        assert py == c
+
+
+def _run_stream(alpha_seq, w, page_size, check_each_step=True):
+    pages = len(alpha_seq) // page_size + 1
+    sim = oracle.Sim(1, 1, w, max_pages=pages, max_pages_per_stream=pages, page_size=page_size)
+    for s, bit in enumerate(alpha_seq):
+        rc, _ = sim.append([0], [1], np.array([[bit]], dtype=np.uint8))
+        assert rc == 0
+        if check_each_step or s == len(alpha_seq) - 1:
+            ret = sim.retained(0).tolist()
+            vis = oracle.visible_positions(alpha_seq, s, w)
+            assert sorted(ret) == vis, (alpha_seq, w, s)
+            assert len(set(ret)) == len(ret)
+            assert len(ret) == oracle.retained_count_closed_form(alpha_seq, s, w)
+            snap = sim.snapshot()
+            assert snap["n_pages"][0] == -(-len(ret) // page_size)
+    return sim
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 8, 10])
+def test_brute_force_all_patterns(T):
+    for w in sorted({1, 2, 3, 5, T}):
+        for bits in itertools.product((0, 1), repeat=T):
+            _run_stream(list(bits), w, page_size=4)
+
+
+def test_brute_force_length12():
+    T = 12
+    for w in (1, 3, 5, 12):
+        for bits in itertools.product((0, 1), repeat=T):
+            _run_stream(list(bits), w, page_size=4, check_each_step=False)
+
+
+def test_bulk_append_equals_token_by_token():
+    rng = np.random.default_rng(3)
+    for w in (1, 4, 16, 37):
+        a = rng.integers(0, 2, (300, 2)).astype(np.uint8)
+        s1 = oracle.Sim(1, 2, w, 64, 64)
+        for t in range(300):
+            assert s1.append([0], [1], a[t:t + 1])[0] == 0
+        s2 = oracle.Sim(1, 2, w, 64, 64)
+        assert s2.append([0], [120], a[:120])[0] == 0
+        assert s2.append([0], [180], a[120:])[0] == 0
+        x, y = s1.snapshot(), s2.snapshot()
+        for k in ("n", "pos", "n_pages"):
+            np.testing.assert_array_equal(x[k], y[k])
+        # page ids differ only in pop order across streams; the retained sets match
+        for st in range(2):
+            assert s1.retained(st).tolist() == s2.retained(st).tolist()
+
+
+def test_closed_form_random_long():
+    rng = np.random.default_rng(11)
+    for w, p in ((256, 0.875), (16, 0.5), (1, 0.3)):
+        a = (rng.random(3000) < p).astype(np.uint8)
+        sim = _run_stream(a.tolist(), w, page_size=16, check_each_step=False)
+        assert sim.snapshot()["n"][0] == oracle.retained_count_closed_form(a, 2999, w)
+
+
+def test_all_marked_keeps_exactly_w():
+    for w in (1, 2, 7, 16):
+        sim = _run_stream([1] * 50, w, page_size=16, check_each_step=False)
+        assert sorted(sim.retained(0).tolist()) == list(range(50 - w, 50))
+
+
+def test_window_covers_context_keeps_all():
+    rng = np.random.default_rng(5)
+    a = rng.integers(0, 2, 40).tolist()
+    sim = _run_stream(a, 40, page_size=16, check_each_step=False)
+    assert sorted(sim.retained(0).tolist()) == list(range(40))
+
+
+def test_golden_page_pops():
+    sim = oracle.Sim(2, 2, 64, max_pages=16, max_pages_per_stream=8)
+    for line in open(os.path.join(GOLD, "page_pops.txt")):
+        line = line.split("#", 1)[0].strip()
+        if not line:
+            continue
+        f = line.split()
+        if f[0] == "op":
+            kw = dict(x.split("=") for x in f[2:])
+            seq = int(kw["seq"])
+            if f[1] == "append":
+                t = int(kw["tokens"])
+                assert sim.append([seq], [t], np.zeros((t, 2), np.uint8))[0] == 0
+            else:
+                assert sim.reset_seq(seq) == 0
+        elif f[0] == "expect":
+            st = int(f[1])
+            pages = [int(x) for x in line.split(":")[1].split()]
+            snap = sim.snapshot()
+            assert snap["n_pages"][st] == len(pages)
+            assert snap["page_table"][st][:len(pages)].tolist() == pages
+        elif f[0] == "free_count":
+            assert sim.snapshot()["free_count"] == int(f[1])
+
+
+def test_pool_exhaustion_and_stream_capacity():
+    sim = oracle.Sim(1, 1, 8, max_pages=2, max_pages_per_stream=8)
+    assert sim.append([0], [32], np.zeros((32, 1), np.uint8))[0] == 0
+    assert sim.append([0], [1], np.zeros((1, 1), np.uint8))[0] == 2   # pool exhausted
+    sim2 = oracle.Sim(1, 1, 8, max_pages=8, max_pages_per_stream=1)
+    assert sim2.append([0], [16], np.zeros((16, 1), np.uint8))[0] == 0
+    assert sim2.append([0], [1], np.zeros((1, 1), np.uint8))[0] == 6
