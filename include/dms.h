@@ -1,0 +1,189 @@
+/*
+ * dms.h - C ABI of libdms: decode-time Dynamic Memory Sparsification (DMS)
+ * over a paged, per-KV-head slot pool on one NVIDIA B200 (sm_100a).
+ *
+ * The method ("Inference-Time Hyper-Scaling with KV Cache Compression",
+ * paper summary, Key claims and Method, section 3.2):
+ *   - every KV head takes a binary eviction decision alpha_t for the token
+ *     it appends at step t;
+ *   - delayed eviction: a token marked at step t stays attendable until
+ *     step t + w (w = 256 by default, section 5.3 and Fig. 5), then leaves;
+ *   - eviction acts as an attention mask that is never materialised, and the
+ *     sparsified cache works with paged KV storage (section 3.2
+ *     "Performance Considerations", section 3.3).
+ * Reading of the window bound used throughout: position j is visible to
+ * the query at step s iff alpha_j == 0 or s - j < w.
+ *
+ * Storage. A *stream* is one (sequence, KV head) pair, stream id =
+ * seq_id * num_kv_heads + kv_head. A stream holds its retained tokens in
+ * logical slots [0, n); logical slot l lives in physical page
+ * page_table[stream][l / 16] at row l % 16. A page holds 16 K rows then 16
+ * V rows of head_dim elements each, contiguous. Pages come from one global
+ * free stack (a fresh pool pops 0, 1, 2, ...).
+ * When token s is appended to a stream and s >= w and the token at s - w
+ * was marked, that token leaves now and s takes its logical slot; otherwise
+ * s takes the fresh slot n and n grows by one, popping a page first when n
+ * is a multiple of 16. Hence slots [0, n) are always exactly the retained
+ * tokens and n never shrinks while a sequence lives.
+ * Within one append call, streams take pages in (order of seq_ids in the
+ * call, KV head ascending) order.
+ *
+ * Conventions.
+ *   - Every tensor argument is caller-owned DEVICE memory on the cache's
+ *     device, row-major and contiguous, unless stated otherwise.
+ *   - Calls enqueue work on the caller's stream and return without
+ *     synchronising, except where stated ("syncs").
+ *   - Errors found on the host (bad arguments, CUDA launch failures) are
+ *     returned at once. Errors found on the device (pool exhausted, stream
+ *     full, bad sequence id, bounded-wait timeout) latch into a status word
+ *     and *poison* the cache: every later kernel on it does nothing until
+ *     dms_cache_reset. Read the word with dms_get_status (syncs).
+ *   - One cache must not be used from two streams at the same time. Calls
+ *     on one stream run in order; dms_append of a step must precede the
+ *     dms_decode_attention that should see that step's token.
+ *   - seq_ids inside one call must be distinct.
+ */
+#ifndef DMS_H
+#define DMS_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct dms_cache dms_cache;   /* opaque, owned by the library */
+
+typedef enum {
+    DMS_OK = 0,
+    DMS_ERR_INVALID = 1,          /* bad argument or configuration */
+    DMS_ERR_POOL_EXHAUSTED = 2,   /* free page stack empty (device) */
+    DMS_ERR_CUDA = 3,             /* a CUDA call failed */
+    DMS_ERR_TIMEOUT = 4,          /* a bounded wait inside a kernel ran out (device) */
+    DMS_ERR_POISONED = 5,         /* host calls refuse work once dms_get_status saw a device error */
+    DMS_ERR_STREAM_FULL = 6,      /* a stream would exceed max_pages_per_stream (device) */
+    DMS_ERR_BAD_SEQ = 7           /* a device-side seq_id outside [0, max_seqs) (device) */
+} dms_status;
+
+typedef enum { DMS_BF16 = 0, DMS_F32 = 1 } dms_dtype;
+
+typedef enum {
+    DMS_ATTN_AUTO = 0,   /* tensor-core page kernel for bf16, CUDA-core kernel for f32 */
+    DMS_ATTN_SIMT = 1,   /* CUDA-core kernel: warp-shuffle dot products, any dtype */
+    DMS_ATTN_MMA = 2     /* mma.sync m16n8k16 page kernel (bf16 only, GQA group <= 8) */
+} dms_attn_kernel;
+
+typedef struct {
+    int32_t max_seqs;              /* sequences the cache can hold (seq_id in [0, max_seqs)) */
+    int32_t num_kv_heads;          /* KV heads per sequence; max_seqs * num_kv_heads <= 8192 */
+    int32_t head_dim;              /* 64 or 128 */
+    int32_t page_size;             /* must be 16 */
+    int32_t window;                /* delayed-eviction window w >= 1 */
+    int32_t max_pages;             /* pages in the shared pool, 1 .. 2^27 */
+    int32_t max_pages_per_stream;  /* page-table length of one stream */
+    dms_dtype dtype;               /* storage type of K, V (and Q) */
+    dms_attn_kernel attn_kernel;   /* decode-attention kernel choice */
+} dms_config;
+
+/* Create a cache on the current CUDA device. Allocates the pool
+ * (max_pages * 2 * 16 * head_dim elements), the page tables, the free stack,
+ * the per-stream counters and window rings, and the split-K scratch
+ * (partials and per-stream counters). Zeroes everything. Syncs.
+ * Returns DMS_ERR_INVALID for an unsupported configuration, DMS_ERR_CUDA if
+ * an allocation fails (nothing leaks). */
+dms_status dms_cache_create(const dms_config* cfg, dms_cache** out);
+
+/* Free everything. Syncs the device. NULL is accepted. */
+dms_status dms_cache_destroy(dms_cache* cache);
+
+/* Return the cache to its freshly created state (all sequences empty, free
+ * stack full, status cleared). Pool contents are not cleared. Async. */
+dms_status dms_cache_reset(dms_cache* cache, cudaStream_t stream);
+
+/* Release sequence seq_id (host int): push its pages back on the free stack
+ * (KV head ascending, each stream's pages last to first) and clear its
+ * counters and window rings. Async. */
+dms_status dms_seq_reset(dms_cache* cache, cudaStream_t stream, int32_t seq_id);
+
+/* Append tokens and apply delayed eviction (paper summary, Method; section
+ * 3.2). For every (sequence, KV head) stream of the call and every new token
+ * s in position order: retire the token at s - w if it was marked and reuse
+ * its slot, else take a fresh slot; write the K and V rows into the pool;
+ * record alpha_s.
+ *   n_seqs        sequences in this call (host int, >= 0)
+ *   seq_ids       device int32 [n_seqs], distinct, each in [0, max_seqs)
+ *   cu_tokens     device int32 [n_seqs + 1] prefix offsets of each
+ *                 sequence's tokens, or NULL for exactly one token per
+ *                 sequence (the decode step; total_tokens must be n_seqs)
+ *   total_tokens  host int, rows in K, V and alpha
+ *   K, V          device [total_tokens, num_kv_heads, head_dim] of dtype;
+ *                 rows of sequence i are cu_tokens[i] .. cu_tokens[i+1]-1
+ *   alpha         device uint8 [total_tokens, num_kv_heads]; 0 keeps the
+ *                 token, any other value marks it for delayed eviction
+ * Device errors: DMS_ERR_POOL_EXHAUSTED (no page is taken by any stream
+ * that needed one in this call; those streams are left unchanged),
+ * DMS_ERR_STREAM_FULL, DMS_ERR_BAD_SEQ. Async. */
+dms_status dms_append(dms_cache* cache, cudaStream_t stream, int32_t n_seqs,
+                      const int32_t* seq_ids, const int32_t* cu_tokens, int32_t total_tokens,
+                      const void* K, const void* V, const uint8_t* alpha);
+
+/* One decode step of GQA attention over the retained tokens (paper summary,
+ * Key claims: memory reads dominate decode latency; the mask is never
+ * materialised). For each sequence b of the call and query head h:
+ *   out[b, h] = sum_{j retained} softmax_j(scale * Q[b, h] . K_j) V_j
+ * over the retained tokens of stream (seq_ids[b], h / g), g = num_q_heads /
+ * num_kv_heads. Split-K over retained pages with fp32 online softmax; the
+ * partial results are merged inside the same kernel (no second launch).
+ *   seq_ids      device int32 [n_seqs], distinct
+ *   Q            device [n_seqs, num_q_heads, head_dim] of the cache dtype
+ *   num_q_heads  host int; a multiple of num_kv_heads with g <= 8
+ *   scale        host float (usually 1 / sqrt(head_dim))
+ *   out          device [n_seqs, num_q_heads, head_dim] of out_dtype
+ * A stream with no tokens yields zeros. Async. */
+dms_status dms_decode_attention(dms_cache* cache, cudaStream_t stream, int32_t n_seqs,
+                                const int32_t* seq_ids, const void* Q, int32_t num_q_heads,
+                                float scale, void* out, dms_dtype out_dtype);
+
+/* Retained counts and compression ratios (paper summary, Key claims: CR =
+ * tokens seen / tokens kept; each head can land at its own CR). Async;
+ * every output is device memory and optional (NULL skips it).
+ *   retained  int32 [max_seqs * num_kv_heads]  n of every stream
+ *   seen      int32 [max_seqs * num_kv_heads]  tokens appended to every stream
+ *   head_cr   float [num_kv_heads]   sum(seen) / sum(retained) over all
+ *             sequences for each KV head (0 when nothing is retained)
+ *   totals    int64 [2]              { sum(seen), sum(retained) } */
+dms_status dms_stats(dms_cache* cache, cudaStream_t stream, int32_t* retained, int32_t* seen,
+                     float* head_cr, int64_t* totals);
+
+/* Copy the bookkeeping to HOST memory for checking. Syncs the stream. Any
+ * pointer may be NULL.
+ *   page_table  int32 [S * max_pages_per_stream]   (entries >= n_pages are stale)
+ *   n_pages, n, pos  int32 [S]
+ *   slot_pos    int32 [max_pages * 16]  position stored in each physical slot
+ *               (stale outside a stream's slots [0, n))
+ *   free_list   int32 [max_pages], free_count int32 [1] */
+dms_status dms_snapshot(dms_cache* cache, cudaStream_t stream, int32_t* page_table,
+                        int32_t* n_pages, int32_t* n, int32_t* pos, int32_t* slot_pos,
+                        int32_t* free_list, int32_t* free_count);
+
+/* Gather the retained K and V rows of one stream in logical slot order into
+ * device buffers [n, head_dim] of the cache dtype (n from dms_stats or
+ * dms_snapshot; rows_cap bounds the copy). Async. */
+dms_status dms_gather_kv(dms_cache* cache, cudaStream_t stream, int32_t seq_id,
+                         int32_t kv_head, int32_t rows_cap, void* K_out, void* V_out);
+
+/* Sync the stream and return the latched device status (DMS_OK if none). */
+dms_status dms_get_status(dms_cache* cache, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char* dms_status_string(dms_status s);
+
+/* Kernel launches issued by the library since the cache was created (host
+ * counter, for accounting). */
+int64_t dms_launch_count(const dms_cache* cache);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DMS_H */

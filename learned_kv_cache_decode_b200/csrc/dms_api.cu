@@ -1,0 +1,258 @@
+// dms_api.cu - the extern "C" boundary of libdms (see include/dms.h).
+//
+// Host code only: argument checks, allocation, and kernel launches on the
+// caller's stream. Every step of the decode path runs in the kernels of
+// dms_append.cu and dms_attention.cu.
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "dms_internal.cuh"
+
+struct dms_cache {
+  dms_config cfg;
+  int device = 0;
+  int num_sms = 0;
+  dms::Dev dv{};
+  dms::AttnPlan plan{};
+  int64_t launches = 0;
+  bool poisoned = false;   // a device error was observed by dms_get_status
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dms_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DMS_OK : DMS_ERR_CUDA; }
+
+// Every call must run with the cache's device current.
+dms_status check_device(const dms_cache* c) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DMS_ERR_CUDA;
+  return dev == c->device ? DMS_OK : DMS_ERR_INVALID;
+}
+
+// Work-issuing calls refuse a cache whose device error has been observed.
+dms_status check_usable(const dms_cache* c) {
+  if (dms_status s = check_device(c)) return s;
+  return c->poisoned ? DMS_ERR_POISONED : DMS_OK;
+}
+
+void free_all(dms::Dev& dv) {
+  void* ptrs[] = {dv.pos, dv.n, dv.n_pages, dv.page_table, dv.ring, dv.slot_pos, dv.free_list,
+                  dv.ctrl, dv.scratch, dv.kv, dv.part, dv.cnt};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  dv = dms::Dev{};
+}
+
+template <typename T>
+cudaError_t alloc(T** p, size_t count) {
+  return cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T) + 16);
+}
+
+}  // namespace
+
+extern "C" {
+
+dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
+  if (!cfg || !out) return DMS_ERR_INVALID;
+  *out = nullptr;
+  const dms_config& c = *cfg;
+  if (c.max_seqs < 1 || c.num_kv_heads < 1 || c.num_kv_heads > dms::kMaxKvHeads) return DMS_ERR_INVALID;
+  if ((int64_t)c.max_seqs * c.num_kv_heads > dms::kMaxStreams) return DMS_ERR_INVALID;
+  if (c.head_dim != 64 && c.head_dim != 128) return DMS_ERR_INVALID;
+  if (c.page_size != dms::kPage || c.window < 1) return DMS_ERR_INVALID;
+  if (c.max_pages < 1 || c.max_pages > (1 << 27) || c.max_pages_per_stream < 1) return DMS_ERR_INVALID;
+  if (c.dtype != DMS_BF16 && c.dtype != DMS_F32) return DMS_ERR_INVALID;
+  if (c.attn_kernel != DMS_ATTN_AUTO && c.attn_kernel != DMS_ATTN_SIMT && c.attn_kernel != DMS_ATTN_MMA)
+    return DMS_ERR_INVALID;
+  if (c.attn_kernel == DMS_ATTN_MMA && c.dtype != DMS_BF16) return DMS_ERR_INVALID;
+  if ((int64_t)c.max_seqs * c.num_kv_heads * c.window > (int64_t)1 << 31) return DMS_ERR_INVALID;
+  if ((int64_t)c.max_seqs * c.num_kv_heads * c.max_pages_per_stream > (int64_t)1 << 31) return DMS_ERR_INVALID;
+
+  dms_cache* h = new (std::nothrow) dms_cache();
+  if (!h) return DMS_ERR_CUDA;
+  h->cfg = c;
+  if (cudaGetDevice(&h->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+    delete h;
+    return DMS_ERR_CUDA;
+  }
+  dms::Dev& dv = h->dv;
+  dv.S = c.max_seqs * c.num_kv_heads;
+  dv.hkv = c.num_kv_heads;
+  dv.d = c.head_dim;
+  dv.w = c.window;
+  dv.mps = c.max_pages_per_stream;
+  dv.max_pages = c.max_pages;
+  dv.max_seqs = c.max_seqs;
+  dv.elem_bytes = c.dtype == DMS_BF16 ? 2 : 4;
+
+  const size_t S = dv.S;
+  cudaError_t e = cudaSuccess;
+  auto step = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
+  step(alloc(&dv.pos, S));
+  step(alloc(&dv.n, S));
+  step(alloc(&dv.n_pages, S));
+  step(alloc(&dv.page_table, S * dv.mps));
+  step(alloc(&dv.ring, S * dv.w));
+  step(alloc(&dv.slot_pos, (size_t)dv.max_pages * dms::kPage));
+  step(alloc(&dv.free_list, (size_t)dv.max_pages));
+  step(alloc(&dv.ctrl, (size_t)dms::kCtrlWords));
+  step(alloc(&dv.scratch, S));
+  step(alloc(&dv.cnt, S));
+  step(alloc(&dv.kv, (size_t)dv.max_pages * 2 * dms::kPage * dv.d * dv.elem_bytes));
+  if (e == cudaSuccess) e = dms::attention_prepare(dv, c.dtype, c.attn_kernel, h->num_sms, &h->plan);
+  if (e == cudaSuccess)
+    e = alloc(&dv.part, (size_t)(h->plan.grid + dv.S) * dms::kMaxGroup * (dv.d + 2));
+  if (e == cudaSuccess) e = cudaMemset(dv.kv, 0, (size_t)dv.max_pages * 2 * dms::kPage * dv.d * dv.elem_bytes);
+  if (e == cudaSuccess) e = cudaMemset(dv.page_table, 0xff, S * dv.mps * sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaMemset(dv.slot_pos, 0xff, (size_t)dv.max_pages * dms::kPage * sizeof(int32_t));
+  if (e == cudaSuccess) e = dms::launch_init_state(dv, 0);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    free_all(dv);
+    delete h;
+    cudaGetLastError();
+    return e == cudaErrorInvalidValue ? DMS_ERR_INVALID : DMS_ERR_CUDA;
+  }
+  h->launches = 1;
+  *out = h;
+  return DMS_OK;
+}
+
+dms_status dms_cache_destroy(dms_cache* h) {
+  if (!h) return DMS_OK;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(h->device);
+  cudaError_t e = cudaDeviceSynchronize();
+  free_all(h->dv);
+  if (prev >= 0) cudaSetDevice(prev);
+  delete h;
+  return from_cuda(e);
+}
+
+dms_status dms_cache_reset(dms_cache* h, cudaStream_t stream) {
+  if (!h) return DMS_ERR_INVALID;
+  if (dms_status s = check_device(h)) return s;
+  cudaError_t e = cudaMemsetAsync(h->dv.page_table, 0xff, (size_t)h->dv.S * h->dv.mps * sizeof(int32_t), stream);
+  if (e == cudaSuccess) e = dms::launch_init_state(h->dv, stream);
+  h->launches += 1;
+  if (e == cudaSuccess) h->poisoned = false;
+  return from_cuda(e);
+}
+
+dms_status dms_seq_reset(dms_cache* h, cudaStream_t stream, int32_t seq_id) {
+  if (!h || seq_id < 0 || seq_id >= h->cfg.max_seqs) return DMS_ERR_INVALID;
+  if (dms_status s = check_usable(h)) return s;
+  h->launches += 1;
+  return from_cuda(dms::launch_reset_seq(h->dv, stream, seq_id));
+}
+
+dms_status dms_append(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                      const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
+                      const uint8_t* alpha) {
+  if (!h || n_seqs < 0 || n_seqs > h->cfg.max_seqs || total_tokens < 0) return DMS_ERR_INVALID;
+  if (dms_status s = check_usable(h)) return s;
+  if (n_seqs == 0) return DMS_OK;
+  if (!seq_ids || (total_tokens > 0 && (!K || !V || !alpha))) return DMS_ERR_INVALID;
+  if (!aligned16(K) || !aligned16(V)) return DMS_ERR_INVALID;
+  int launches = 0;
+  cudaError_t e;
+  if (cu_tokens == nullptr) {
+    if (total_tokens != n_seqs) return DMS_ERR_INVALID;
+    e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, &launches);
+  } else {
+    e = dms::launch_append_bulk(h->dv, stream, n_seqs, seq_ids, cu_tokens, total_tokens, K, V, alpha,
+                                &launches);
+  }
+  h->launches += launches;
+  return from_cuda(e);
+}
+
+dms_status dms_decode_attention(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                                const void* Q, int32_t num_q_heads, float scale, void* out,
+                                dms_dtype out_dtype) {
+  if (!h || n_seqs < 0 || n_seqs > h->cfg.max_seqs) return DMS_ERR_INVALID;
+  if (dms_status s = check_usable(h)) return s;
+  if (num_q_heads < h->cfg.num_kv_heads || num_q_heads % h->cfg.num_kv_heads != 0) return DMS_ERR_INVALID;
+  if (num_q_heads / h->cfg.num_kv_heads > dms::kMaxGroup) return DMS_ERR_INVALID;
+  if (out_dtype != DMS_BF16 && out_dtype != DMS_F32) return DMS_ERR_INVALID;
+  if (n_seqs == 0) return DMS_OK;
+  if (!seq_ids || !Q || !out || !aligned16(Q) || !aligned16(out)) return DMS_ERR_INVALID;
+  h->launches += 1;
+  return from_cuda(dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
+                                         out_dtype == DMS_F32));
+}
+
+dms_status dms_stats(dms_cache* h, cudaStream_t stream, int32_t* retained, int32_t* seen, float* head_cr,
+                     int64_t* totals) {
+  if (!h) return DMS_ERR_INVALID;
+  if (dms_status s = check_usable(h)) return s;
+  h->launches += 1;
+  return from_cuda(dms::launch_stats(h->dv, stream, retained, seen, head_cr, totals));
+}
+
+dms_status dms_snapshot(dms_cache* h, cudaStream_t stream, int32_t* page_table, int32_t* n_pages, int32_t* n,
+                        int32_t* pos, int32_t* slot_pos, int32_t* free_list, int32_t* free_count) {
+  if (!h) return DMS_ERR_INVALID;
+  if (dms_status s = check_device(h)) return s;
+  const dms::Dev& dv = h->dv;
+  const size_t S = dv.S;
+  cudaError_t e = cudaSuccess;
+  auto cp = [&](void* dst, const void* src, size_t bytes) {
+    if (dst && e == cudaSuccess) e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, stream);
+  };
+  cp(page_table, dv.page_table, S * dv.mps * sizeof(int32_t));
+  cp(n_pages, dv.n_pages, S * sizeof(int32_t));
+  cp(n, dv.n, S * sizeof(int32_t));
+  cp(pos, dv.pos, S * sizeof(int32_t));
+  cp(slot_pos, dv.slot_pos, (size_t)dv.max_pages * dms::kPage * sizeof(int32_t));
+  cp(free_list, dv.free_list, (size_t)dv.max_pages * sizeof(int32_t));
+  cp(free_count, dv.ctrl + dms::kCtrlFree, sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  return from_cuda(e);
+}
+
+dms_status dms_gather_kv(dms_cache* h, cudaStream_t stream, int32_t seq_id, int32_t kv_head, int32_t rows_cap,
+                         void* K_out, void* V_out) {
+  if (!h || seq_id < 0 || seq_id >= h->cfg.max_seqs || kv_head < 0 || kv_head >= h->cfg.num_kv_heads)
+    return DMS_ERR_INVALID;
+  if (dms_status s = check_usable(h)) return s;
+  if (rows_cap <= 0) return DMS_OK;
+  if (!K_out || !V_out || !aligned16(K_out) || !aligned16(V_out)) return DMS_ERR_INVALID;
+  h->launches += 1;
+  return from_cuda(dms::launch_gather(h->dv, stream, seq_id, kv_head, rows_cap, K_out, V_out));
+}
+
+dms_status dms_get_status(dms_cache* h, cudaStream_t stream) {
+  if (!h) return DMS_ERR_INVALID;
+  if (dms_status s = check_device(h)) return s;
+  int32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, h->dv.ctrl + dms::kCtrlStatus, sizeof(word), cudaMemcpyDeviceToHost,
+                                  stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return DMS_ERR_CUDA;
+  if (word != DMS_OK) h->poisoned = true;
+  return (dms_status)word;
+}
+
+const char* dms_status_string(dms_status s) {
+  switch (s) {
+    case DMS_OK: return "ok";
+    case DMS_ERR_INVALID: return "invalid argument or configuration";
+    case DMS_ERR_POOL_EXHAUSTED: return "page pool exhausted";
+    case DMS_ERR_CUDA: return "CUDA error";
+    case DMS_ERR_TIMEOUT: return "bounded wait timed out inside a kernel";
+    case DMS_ERR_POISONED: return "cache poisoned by an earlier device error";
+    case DMS_ERR_STREAM_FULL: return "stream page table full";
+    case DMS_ERR_BAD_SEQ: return "sequence id out of range";
+  }
+  return "unknown status";
+}
+
+int64_t dms_launch_count(const dms_cache* h) { return h ? h->launches : 0; }
+
+}  // extern "C"

@@ -1,0 +1,469 @@
+// dms_append.cu - cache bookkeeping kernels: decode append, bulk (prefill)
+// append, sequence reset, whole-cache reset, statistics, K/V gather.
+//
+// Retention rule ("Inference-Time Hyper-Scaling with KV Cache Compression",
+// paper summary, Key claims and Method, section 3.2): the decision alpha_t
+// of a token acts w steps later. With the bound read as "visible iff
+// alpha_j == 0 or s - j < w", the token that can leave when token s arrives
+// is exactly s - w, so appending s either reuses the slot of s - w (marked)
+// or takes a fresh slot. Slots [0, n) therefore stay dense and no validity
+// bitmap or mask is ever stored.
+#include "dms_internal.cuh"
+
+namespace dms {
+
+namespace {
+
+constexpr int kDecodeThreads = 128;
+constexpr int kDecodeStreamsPerBlock = 32;
+
+__device__ __forceinline__ uint8_t* page_row(const Dev& dv, int page, int which, int row, int row_bytes) {
+  return dv.kv + ((size_t)page * 2 * kPage + (size_t)which * kPage + row) * row_bytes;
+}
+
+// Copy one K or V row (row_bytes, multiple of 16) with a warp of 16-byte vectors.
+__device__ __forceinline__ void warp_copy_row(uint8_t* dst, const uint8_t* src, int row_bytes, int lane) {
+  const int vec = row_bytes >> 4;
+  for (int v = lane; v < vec; v += 32)
+    reinterpret_cast<uint4*>(dst)[v] = __ldg(reinterpret_cast<const uint4*>(src) + v);
+}
+
+// ---------------------------------------------------------------------------
+// Decode append: one token for each sequence of the call.
+//
+// Every block owns 32 streams (one lane of warp 0 each). A stream whose new
+// token reuses a retired slot or lands inside an already attached page is
+// finished by its own block. A stream whose token opens a new page is left
+// to the last block to arrive, which pops pages for all of them in stream
+// order, so page ids are deterministic without any inter-block waiting.
+__global__ void __launch_bounds__(kDecodeThreads)
+append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
+                     const uint8_t* __restrict__ K, const uint8_t* __restrict__ V,
+                     const uint8_t* __restrict__ alpha) {
+  __shared__ int s_phys[kDecodeStreamsPerBlock];
+  __shared__ int s_warp[kDecodeThreads / 32];
+  __shared__ int s_last, s_ok;
+  const int nst = n_seqs * dv.hkv;
+  const int row_bytes = dv.d * dv.elem_bytes;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i0 = blockIdx.x * kDecodeStreamsPerBlock;
+  if (tid == 0) s_ok = (read_status(dv.ctrl) == 0);
+  __syncthreads();
+  const bool ok = s_ok;
+
+  if (tid < kDecodeStreamsPerBlock) {
+    const int i = i0 + tid;
+    int phys = -1;
+    if (ok && i < nst) {
+      int need = 0;
+      const int seq = seq_ids[i / dv.hkv];
+      if (seq < 0 || seq >= dv.max_seqs) {
+        latch(dv.ctrl, DMS_ERR_BAD_SEQ);
+      } else {
+        const int st = seq * dv.hkv + i % dv.hkv;
+        const int s = dv.pos[st];
+        int32_t* rp = dv.ring + (size_t)st * dv.w + (s % dv.w);
+        const int r = *rp;
+        const bool retire = (s >= dv.w) && (r & 1);   // token s - w leaves now
+        const int slot = retire ? (r >> 1) : dv.n[st];
+        if (!retire && (slot % kPage) == 0) {
+          need = 1;   // opens a page: finished by the last block
+        } else {
+          const int page = slot / kPage < dv.mps ? dv.page_table[(size_t)st * dv.mps + slot / kPage] : -1;
+          if (page < 0 || page >= dv.max_pages) {
+            latch(dv.ctrl, DMS_ERR_INVALID);
+          } else {
+            if (!retire) dv.n[st] = slot + 1;
+            phys = page * kPage + slot % kPage;
+            *rp = (slot << 1) | (alpha[i] != 0);
+            dv.pos[st] = s + 1;
+            dv.slot_pos[phys] = s;
+          }
+        }
+      }
+      dv.scratch[i] = need;
+    }
+    s_phys[tid] = phys;
+  }
+  __syncthreads();
+
+  // K and V rows of the streams finished here (warp per stream).
+  for (int l = warp; l < kDecodeStreamsPerBlock; l += kDecodeThreads / 32) {
+    const int phys = s_phys[l];
+    if (phys < 0) continue;
+    const size_t src = (size_t)(i0 + l) * row_bytes;
+    warp_copy_row(page_row(dv, phys / kPage, 0, phys % kPage, row_bytes), K + src, row_bytes, lane);
+    warp_copy_row(page_row(dv, phys / kPage, 1, phys % kPage, row_bytes), V + src, row_bytes, lane);
+  }
+
+  // Last block to arrive pops pages for the deferred streams.
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&dv.ctrl[kCtrlArrive], 1) == (int)gridDim.x - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  const bool still_ok = ok && read_status(dv.ctrl) == 0;
+  const int per = (nst + kDecodeThreads - 1) / kDecodeThreads;
+  const int b = min(tid * per, nst), e = min(b + per, nst);
+  int cnt = 0;
+  if (still_ok)
+    for (int i = b; i < e; ++i) cnt += __ldcg(&dv.scratch[i]);
+  int total;
+  int rank = block_exclusive_scan(cnt, s_warp, &total);
+  const int fc = *reinterpret_cast<volatile int32_t*>(&dv.ctrl[kCtrlFree]);
+  const bool fits = still_ok && total <= fc;
+  if (still_ok && !fits && tid == 0) latch(dv.ctrl, DMS_ERR_POOL_EXHAUSTED);
+  if (fits && total > 0) {
+    for (int i = b; i < e; ++i) {
+      if (__ldcg(&dv.scratch[i]) == 0) continue;
+      const int page = dv.free_list[fc - 1 - rank];
+      ++rank;
+      const int st = seq_ids[i / dv.hkv] * dv.hkv + i % dv.hkv;
+      const int s = dv.pos[st];
+      const int slot = dv.n[st];
+      const int lp = slot / kPage;
+      if (lp >= dv.mps) {
+        latch(dv.ctrl, DMS_ERR_STREAM_FULL);
+        dv.scratch[i] = 0;
+        continue;
+      }
+      dv.page_table[(size_t)st * dv.mps + lp] = page;
+      dv.n_pages[st] = lp + 1;
+      dv.n[st] = slot + 1;
+      dv.ring[(size_t)st * dv.w + (s % dv.w)] = (slot << 1) | (alpha[i] != 0);
+      dv.pos[st] = s + 1;
+      dv.slot_pos[page * kPage] = s;
+      dv.scratch[i] = -(page + 1);   // row copy below
+    }
+  }
+  __syncthreads();
+  if (fits && total > 0) {
+    // Copy rows of the deferred streams, warp per stream.
+    for (int base = warp * 32; base < nst; base += kDecodeThreads) {
+      const int i = base + lane;
+      const int v = (i < nst) ? __ldcg(&dv.scratch[i]) : 0;
+      unsigned mask = __ballot_sync(0xffffffffu, v < 0);
+      while (mask) {
+        const int l = __ffs(mask) - 1;
+        mask &= mask - 1;
+        const int page = -__shfl_sync(0xffffffffu, v, l) - 1;
+        const size_t src = (size_t)(base + l) * row_bytes;
+        warp_copy_row(page_row(dv, page, 0, 0, row_bytes), K + src, row_bytes, lane);
+        warp_copy_row(page_row(dv, page, 1, 0, row_bytes), V + src, row_bytes, lane);
+      }
+    }
+  }
+  if (tid == 0) {
+    if (fits) dv.ctrl[kCtrlFree] = fc - total;
+    dv.ctrl[kCtrlArrive] = 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Bulk append, pass 1: fresh slots each stream will take -> pages it needs.
+// A token j of the call is non-retiring unless j >= w and the token j - w
+// (from this call's alpha, or from the window ring for earlier tokens) was
+// marked.
+__global__ void __launch_bounds__(256)
+bulk_count_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
+                  const int32_t* __restrict__ cu, int total_tokens, const uint8_t* __restrict__ alpha) {
+  __shared__ int s_warp[8];
+  const int i = blockIdx.x;
+  if (read_status(dv.ctrl) != 0) return;
+  const int bseq = i / dv.hkv, kvh = i % dv.hkv;
+  const int seq = seq_ids[bseq];
+  const int t0 = cu[bseq], T = cu[bseq + 1] - t0;
+  if (seq < 0 || seq >= dv.max_seqs) {
+    if (threadIdx.x == 0) { latch(dv.ctrl, DMS_ERR_BAD_SEQ); dv.scratch[i] = 0; }
+    return;
+  }
+  if (t0 < 0 || T < 0 || t0 + T > total_tokens) {
+    if (threadIdx.x == 0) { latch(dv.ctrl, DMS_ERR_INVALID); dv.scratch[i] = 0; }
+    return;
+  }
+  const int st = seq * dv.hkv + kvh;
+  const int s0 = dv.pos[st];
+  int fresh = 0;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const int j = s0 + t;
+    int marked = 0;
+    if (j >= dv.w) {
+      const int jp = j - dv.w;
+      marked = (jp >= s0) ? (alpha[(size_t)(t0 + jp - s0) * dv.hkv + kvh] != 0)
+                          : (dv.ring[(size_t)st * dv.w + jp % dv.w] & 1);
+    }
+    fresh += !marked;
+  }
+  int total;
+  block_exclusive_scan(fresh, s_warp, &total);
+  if (threadIdx.x == 0) {
+    const int n_final = dv.n[st] + total;
+    const int pages = (n_final + kPage - 1) / kPage;
+    if (pages > dv.mps) {
+      latch(dv.ctrl, DMS_ERR_STREAM_FULL);
+      dv.scratch[i] = 0;
+    } else {
+      dv.scratch[i] = pages - dv.n_pages[st];
+    }
+  }
+}
+
+// Bulk append, pass 2 (one block): pop the pages in stream order.
+__global__ void __launch_bounds__(256)
+bulk_pages_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids) {
+  __shared__ int s_warp[8];
+  if (read_status(dv.ctrl) != 0) return;
+  const int nst = n_seqs * dv.hkv;
+  const int per = (nst + blockDim.x - 1) / blockDim.x;
+  const int b = min((int)threadIdx.x * per, nst), e = min(b + per, nst);
+  int cnt = 0;
+  for (int i = b; i < e; ++i) cnt += dv.scratch[i];
+  int total;
+  int rank = block_exclusive_scan(cnt, s_warp, &total);
+  const int fc = dv.ctrl[kCtrlFree];
+  if (total > fc) {
+    if (threadIdx.x == 0) latch(dv.ctrl, DMS_ERR_POOL_EXHAUSTED);
+    return;
+  }
+  for (int i = b; i < e; ++i) {
+    const int k = dv.scratch[i];
+    if (k == 0) continue;
+    const int st = seq_ids[i / dv.hkv] * dv.hkv + i % dv.hkv;
+    const int np0 = dv.n_pages[st];
+    for (int q = 0; q < k; ++q)
+      dv.page_table[(size_t)st * dv.mps + np0 + q] = dv.free_list[fc - 1 - (rank + q)];
+    rank += k;
+    dv.n_pages[st] = np0 + k;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) dv.ctrl[kCtrlFree] = fc - total;
+}
+
+// Bulk append, pass 3: slots, window ring, slot tags and rows, one block per
+// stream. Tokens go in sub-chunks of at most w consecutive positions, so the
+// token j - w every position depends on was settled by an earlier sub-chunk
+// (or lives in the ring). Tokens that leave again within this call (marked
+// and j + w <= last position) are not copied: their slot is overwritten.
+__global__ void __launch_bounds__(256)
+bulk_write_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
+                  const int32_t* __restrict__ cu, const uint8_t* __restrict__ K,
+                  const uint8_t* __restrict__ V, const uint8_t* __restrict__ alpha) {
+  __shared__ int s_warp[8];
+  __shared__ int s_phys[256];
+  if (read_status(dv.ctrl) != 0) return;
+  const int i = blockIdx.x;
+  const int bseq = i / dv.hkv, kvh = i % dv.hkv;
+  const int st = seq_ids[bseq] * dv.hkv + kvh;
+  const int t0 = cu[bseq], T = cu[bseq + 1] - t0;
+  const int s0 = dv.pos[st];
+  const int s_last = s0 + T - 1;
+  const int row_bytes = dv.d * dv.elem_bytes;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int sub = min((int)blockDim.x, dv.w);
+  int n_cur = dv.n[st];
+  int32_t* ring = dv.ring + (size_t)st * dv.w;
+  const int32_t* pt = dv.page_table + (size_t)st * dv.mps;
+
+  for (int c0 = 0; c0 < T; c0 += sub) {
+    const int t = c0 + tid;
+    const bool active = tid < sub && t < T;
+    const int j = s0 + t;
+    int r = 0;
+    bool retire = false;
+    if (active) {
+      r = ring[j % dv.w];
+      retire = (j >= dv.w) && (r & 1);
+    }
+    int total;
+    const int pre = block_exclusive_scan(active && !retire ? 1 : 0, s_warp, &total);
+    int phys = -1;
+    if (active) {
+      const int slot = retire ? (r >> 1) : n_cur + pre;
+      const int a = alpha[(size_t)(t0 + t) * dv.hkv + kvh] != 0;
+      ring[j % dv.w] = (slot << 1) | a;
+      const bool dead = a && (j + dv.w <= s_last);
+      const int page = slot / kPage < dv.mps ? pt[slot / kPage] : -1;
+      if (page < 0 || page >= dv.max_pages) {
+        latch(dv.ctrl, DMS_ERR_INVALID);
+      } else if (!dead) {
+        phys = page * kPage + slot % kPage;
+        dv.slot_pos[phys] = j;
+      }
+    }
+    if (tid < 256) s_phys[tid] = phys;
+    n_cur += total;
+    __syncthreads();
+    const int cnt = min(sub, T - c0);
+    for (int l = warp; l < cnt; l += nw) {
+      const int p = s_phys[l];
+      if (p < 0) continue;
+      const size_t src = ((size_t)(t0 + c0 + l) * dv.hkv + kvh) * row_bytes;
+      warp_copy_row(page_row(dv, p / kPage, 0, p % kPage, row_bytes), K + src, row_bytes, lane);
+      warp_copy_row(page_row(dv, p / kPage, 1, p % kPage, row_bytes), V + src, row_bytes, lane);
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    dv.n[st] = n_cur;
+    dv.pos[st] = s0 + T;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Sequence reset (one block): push pages back, KV head ascending, each
+// stream's pages last to first; clear counters and rings.
+__global__ void __launch_bounds__(256) reset_seq_kernel(Dev dv, int seq) {
+  __shared__ int s_off[kMaxKvHeads + 1];
+  __shared__ int s_fc, s_ok;
+  if (threadIdx.x == 0) {
+    s_ok = read_status(dv.ctrl) == 0;
+    int acc = 0;
+    for (int k = 0; k < dv.hkv; ++k) {
+      s_off[k] = acc;
+      acc += dv.n_pages[seq * dv.hkv + k];
+    }
+    s_off[dv.hkv] = acc;
+    s_fc = dv.ctrl[kCtrlFree];
+    if (s_ok && s_fc + acc > dv.max_pages) {
+      latch(dv.ctrl, DMS_ERR_INVALID);
+      s_ok = 0;
+    }
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  for (int k = 0; k < dv.hkv; ++k) {
+    const int st = seq * dv.hkv + k;
+    const int np = s_off[k + 1] - s_off[k];
+    for (int p = threadIdx.x; p < np; p += blockDim.x)
+      dv.free_list[s_fc + s_off[k] + (np - 1 - p)] = dv.page_table[(size_t)st * dv.mps + p];
+    for (int r = threadIdx.x; r < dv.w; r += blockDim.x) dv.ring[(size_t)st * dv.w + r] = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < dv.hkv; ++k) {
+      const int st = seq * dv.hkv + k;
+      dv.n[st] = 0;
+      dv.pos[st] = 0;
+      dv.n_pages[st] = 0;
+    }
+    dv.ctrl[kCtrlFree] = s_fc + s_off[dv.hkv];
+  }
+}
+
+// Whole-cache reset: fresh free stack (pops 0, 1, 2, ...), empty streams.
+__global__ void init_state_kernel(Dev dv) {
+  const size_t tid = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  const size_t nthr = (size_t)gridDim.x * blockDim.x;
+  for (size_t k = tid; k < (size_t)dv.max_pages; k += nthr) dv.free_list[k] = dv.max_pages - 1 - (int)k;
+  for (size_t k = tid; k < (size_t)dv.S; k += nthr) {
+    dv.pos[k] = 0;
+    dv.n[k] = 0;
+    dv.n_pages[k] = 0;
+    dv.scratch[k] = 0;
+    dv.cnt[k] = 0;
+  }
+  for (size_t k = tid; k < (size_t)dv.S * dv.w; k += nthr) dv.ring[k] = 0;
+  if (tid == 0) {
+    dv.ctrl[kCtrlStatus] = 0;
+    dv.ctrl[kCtrlFree] = dv.max_pages;
+    for (int k = 2; k < kCtrlWords; ++k) dv.ctrl[k] = 0;
+  }
+}
+
+// Statistics (one block).
+__global__ void __launch_bounds__(256)
+stats_kernel(Dev dv, int32_t* retained, int32_t* seen, float* head_cr, int64_t* totals) {
+  __shared__ unsigned long long s_head[kMaxKvHeads][2];
+  for (int h = threadIdx.x; h < dv.hkv; h += blockDim.x) s_head[h][0] = s_head[h][1] = 0;
+  __syncthreads();
+  for (int st = threadIdx.x; st < dv.S; st += blockDim.x) {
+    const int r = dv.n[st], p = dv.pos[st];
+    if (retained) retained[st] = r;
+    if (seen) seen[st] = p;
+    atomicAdd(&s_head[st % dv.hkv][0], (unsigned long long)p);
+    atomicAdd(&s_head[st % dv.hkv][1], (unsigned long long)r);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long a = 0, b = 0;
+    for (int h = 0; h < dv.hkv; ++h) {
+      a += s_head[h][0];
+      b += s_head[h][1];
+      if (head_cr) head_cr[h] = s_head[h][1] ? (float)((double)s_head[h][0] / (double)s_head[h][1]) : 0.f;
+    }
+    if (totals) {
+      totals[0] = (int64_t)a;
+      totals[1] = (int64_t)b;
+    }
+  }
+}
+
+// Gather the retained rows of one stream in logical slot order (warp per row).
+__global__ void __launch_bounds__(256)
+gather_kernel(Dev dv, int seq, int kvh, int rows_cap, uint8_t* Kout, uint8_t* Vout) {
+  const int st = seq * dv.hkv + kvh;
+  const int rows = min(dv.n[st], rows_cap);
+  const int row_bytes = dv.d * dv.elem_bytes;
+  const int lane = threadIdx.x & 31;
+  for (int l = blockIdx.x * 8 + (threadIdx.x >> 5); l < rows; l += gridDim.x * 8) {
+    const int page = dv.page_table[(size_t)st * dv.mps + l / kPage];
+    if (page < 0 || page >= dv.max_pages) continue;
+    warp_copy_row(Kout + (size_t)l * row_bytes, page_row(dv, page, 0, l % kPage, row_bytes), row_bytes, lane);
+    warp_copy_row(Vout + (size_t)l * row_bytes, page_row(dv, page, 1, l % kPage, row_bytes), row_bytes, lane);
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+
+cudaError_t launch_init_state(const Dev& dv, cudaStream_t st) {
+  init_state_kernel<<<256, 256, 0, st>>>(dv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
+                                 const void* K, const void* V, const uint8_t* alpha, int* launches) {
+  const int nst = n_seqs * dv.hkv;
+  if (nst == 0) return cudaSuccess;
+  const int blocks = (nst + kDecodeStreamsPerBlock - 1) / kDecodeStreamsPerBlock;
+  append_decode_kernel<<<blocks, kDecodeThreads, 0, st>>>(dv, n_seqs, seq_ids, (const uint8_t*)K,
+                                                         (const uint8_t*)V, alpha);
+  *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_bulk(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
+                               const int32_t* cu_tokens, int total_tokens, const void* K, const void* V,
+                               const uint8_t* alpha, int* launches) {
+  const int nst = n_seqs * dv.hkv;
+  if (nst == 0) return cudaSuccess;
+  bulk_count_kernel<<<nst, 256, 0, st>>>(dv, n_seqs, seq_ids, cu_tokens, total_tokens, alpha);
+  bulk_pages_kernel<<<1, 256, 0, st>>>(dv, n_seqs, seq_ids);
+  bulk_write_kernel<<<nst, 256, 0, st>>>(dv, n_seqs, seq_ids, cu_tokens, (const uint8_t*)K,
+                                        (const uint8_t*)V, alpha);
+  *launches += 3;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reset_seq(const Dev& dv, cudaStream_t st, int seq) {
+  reset_seq_kernel<<<1, 256, 0, st>>>(dv, seq);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats(const Dev& dv, cudaStream_t st, int32_t* retained, int32_t* seen, float* head_cr,
+                         int64_t* totals) {
+  stats_kernel<<<1, 256, 0, st>>>(dv, retained, seen, head_cr, totals);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const Dev& dv, cudaStream_t st, int seq, int kvh, int rows_cap, void* Kout,
+                          void* Vout) {
+  const int blocks = max(1, min(1024, (rows_cap + 7) / 8));
+  gather_kernel<<<blocks, 256, 0, st>>>(dv, seq, kvh, rows_cap, (uint8_t*)Kout, (uint8_t*)Vout);
+  return cudaGetLastError();
+}
+
+}  // namespace dms

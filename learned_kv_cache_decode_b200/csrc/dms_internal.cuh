@@ -1,0 +1,231 @@
+// dms_internal.cuh - device state and PTX helpers shared by the libdms kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dms.h"
+
+namespace dms {
+
+constexpr int kPage = 16;          // tokens per page
+constexpr int kMaxGroup = 8;       // query heads per KV head handled by one kernel pass
+constexpr int kMaxStreams = 8192;  // max_seqs * num_kv_heads
+constexpr int kMaxKvHeads = 256;
+
+// Control words (device int32).
+enum : int {
+  kCtrlStatus = 0,   // latched dms_status, 0 = healthy
+  kCtrlFree = 1,     // free-stack depth
+  kCtrlArrive = 2,   // arrival counter of the decode-append kernel
+  kCtrlWords = 8
+};
+
+// Everything a kernel needs to know about one cache (device pointers and sizes).
+struct Dev {
+  int32_t* pos;         // [S] tokens seen
+  int32_t* n;           // [S] retained tokens = logical slots in use
+  int32_t* n_pages;     // [S]
+  int32_t* page_table;  // [S][mps]
+  int32_t* ring;        // [S][w] (logical slot << 1) | alpha of the latest token per residue mod w
+  int32_t* slot_pos;    // [max_pages * 16] position held by each physical slot
+  int32_t* free_list;   // [max_pages] stack, top at ctrl[kCtrlFree] - 1
+  int32_t* ctrl;        // [kCtrlWords]
+  int32_t* scratch;     // [S] per-call scratch (append bookkeeping)
+  uint8_t* kv;          // [max_pages][2][16][d] elements: 16 K rows then 16 V rows per page
+  float* part;          // split-K partials [(grid + S)][8][d + 2]
+  int32_t* cnt;         // [S] split-K arrival counters
+  int S, hkv, d, w, mps, max_pages, max_seqs, elem_bytes;
+};
+
+__device__ __forceinline__ void latch(int32_t* ctrl, int code) {
+  atomicCAS(&ctrl[kCtrlStatus], 0, code);
+}
+__device__ __forceinline__ int read_status(const int32_t* ctrl) {
+  return *reinterpret_cast<const volatile int32_t*>(&ctrl[kCtrlStatus]);
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide exclusive scan of one int per thread. `warp_tot` must hold
+// blockDim.x / 32 ints of shared memory. Returns the exclusive prefix and
+// writes the block total to *total. Contains __syncthreads().
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  int before = 0, all = 0;
+  for (int k = 0; k < nw; ++k) {
+    int t = warp_tot[k];
+    if (k < warp) before += t;
+    all += t;
+  }
+  __syncthreads();
+  *total = all;
+  return before + x - v;
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers (sm_90+ / sm_100a). Hand-written; no library code.
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase. Gives up after ~2^31 SM cycles (about a
+// second), latches DMS_ERR_TIMEOUT and raises the CTA's abort flag. Returns
+// false if the data must not be used.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort_flag, int32_t* ctrl) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > (1ll << 31)) {
+      latch(ctrl, DMS_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// Wait with a time bound only (used to drain copies in flight before exit).
+__device__ __forceinline__ void mbar_wait_timed(uint32_t bar, uint32_t parity, int32_t* ctrl) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > (1ll << 31)) {
+      latch(ctrl, DMS_ERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
+// TMA tiled load of a 3-D box into shared memory, completing on an mbarrier.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// Untiled bulk copy global -> shared (size and both addresses 16-B aligned).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// D += A(16x16, row) * B(16x8, col), bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 b16 matrix held in mma fragment layout across the warp.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Hardware base-2 exponential (MUFU). ex2(-inf) = +0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (defined in dms_append.cu / dms_attention.cu).
+
+cudaError_t launch_init_state(const Dev& dv, cudaStream_t st);
+cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
+                                 const void* K, const void* V, const uint8_t* alpha, int* launches);
+cudaError_t launch_append_bulk(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
+                               const int32_t* cu_tokens, int total_tokens, const void* K, const void* V,
+                               const uint8_t* alpha, int* launches);
+cudaError_t launch_reset_seq(const Dev& dv, cudaStream_t st, int seq);
+cudaError_t launch_stats(const Dev& dv, cudaStream_t st, int32_t* retained, int32_t* seen, float* head_cr,
+                         int64_t* totals);
+cudaError_t launch_gather(const Dev& dv, cudaStream_t st, int seq, int kvh, int rows_cap, void* Kout,
+                          void* Vout);
+
+// Decode attention plan shared by host and launcher.
+struct AttnPlan {
+  int kernel;        // DMS_ATTN_SIMT or DMS_ATTN_MMA
+  int grid;          // persistent CTAs
+  int threads;
+  size_t smem;       // dynamic shared memory bytes
+  CUtensorMap tmap;  // pool view for the tiled TMA loads (MMA kernel)
+};
+
+cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan);
+cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,
+                             const int32_t* seq_ids, const void* Q, int hq, float scale, void* out,
+                             int out_f32);
+
+}  // namespace dms

@@ -1,0 +1,212 @@
+"""CUDA path vs the CPU oracle on small seeded cases (GPU).
+
+Each case spans several pages and split-K pieces, ragged last pages and
+sequences of very different lengths. Metadata (page tables, counters, free
+stack, retained sets) must match the oracle's simulator bit for bit;
+outputs must be within max abs 2e-2 / mean abs 2e-3 of the fp64 oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from learned_kv_cache_decode_b200 import workloads as W
+from learned_kv_cache_decode_b200 import _native
+from harness import Run, compare
+
+pytestmark = pytest.mark.gpu
+
+
+def wl(name, batch, hq, hkv, d, dtype, w, ctx_range, steps, p, seed):
+    return W.Workload(name, batch, hq, hkv, d, dtype, w, 0, ctx_range, steps, "bernoulli", (p,), seed)
+
+
+CASES = [
+    wl("f32-g4-d64", 2, 8, 2, 64, "f32", 16, (1, 300), 5, 0.5, 11),
+    wl("f32-g7-d128", 2, 14, 2, 128, "f32", 16, (30, 400), 4, 0.5, 12),
+    wl("bf16-g7-d128", 3, 14, 2, 128, "bf16", 16, (1, 700), 5, 0.6, 13),
+    wl("bf16-g4-d64", 3, 8, 2, 64, "bf16", 64, (100, 900), 5, 0.7, 14),
+    wl("bf16-g5-d128-w1", 2, 10, 2, 128, "bf16", 1, (0, 200), 4, 0.5, 15),
+    wl("bf16-g8-d64", 2, 16, 2, 64, "bf16", 32, (17, 500), 4, 0.9, 16),
+    wl("bf16-g1-d128", 3, 3, 3, 128, "bf16", 8, (5, 90), 4, 0.3, 17),
+    wl("bf16-g2-d64-dense", 2, 4, 2, 64, "bf16", 16, (40, 600), 4, 0.0, 18),
+    wl("bf16-g4-d128-window", 2, 8, 2, 128, "bf16", 48, (40, 600), 4, 1.0, 19),
+    wl("bf16-g7-d128-wide-window", 2, 14, 2, 128, "bf16", 4096, (100, 700), 4, 0.5, 20),
+]
+
+
+def kernels_for(w):
+    return ["simt"] if w.dtype == "f32" else ["mma", "simt"]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c.name for c in CASES])
+def test_small_cases(case):
+    for kern in kernels_for(case):
+        run = Run(case, attn_kernel=kern)
+        try:
+            run.prefill(chunk=97)    # several bulk calls per sequence, odd sizes
+            run.check_metadata()
+            for step in range(case.decode_steps):
+                out, Q = run.decode_step(step)
+                torch.cuda.synchronize()
+                for b in range(case.batch):
+                    ref = run.oracle_out(b, Q[b])
+                    tol = dict(max_abs=1e-4, mean_abs=1e-5) if case.dtype == "f32" else {}
+                    compare(out[b], ref, **tol)
+            run.check_metadata()
+            assert run.cache.status() == _native.DMS_OK
+        finally:
+            run.close()
+
+
+def test_kv_rows_are_copied_bit_exactly():
+    case = wl("gather", 2, 8, 2, 128, "bf16", 16, (200, 300), 3, 0.5, 21)
+    run = Run(case)
+    try:
+        run.prefill(chunk=64)
+        for step in range(3):
+            run.decode_step(step)
+        for b in range(case.batch):
+            T = int(run.seen[b])
+            K, V = W.kv(case, b, 0, T)
+            for h in range(case.num_kv_heads):
+                pos = run.sim.retained(b * case.num_kv_heads + h)
+                gk, gv = run.cache.gather_kv(b, h, len(pos))
+                gk = gk.view(torch.int16).cpu().numpy().view(np.uint16)
+                gv = gv.view(torch.int16).cpu().numpy().view(np.uint16)
+                np.testing.assert_array_equal(gk, K[pos, h])
+                np.testing.assert_array_equal(gv, V[pos, h])
+    finally:
+        run.close()
+
+
+def test_stats_match_oracle_counts():
+    case = wl("stats", 4, 8, 2, 64, "bf16", 16, (10, 500), 2, 0.6, 22)
+    run = Run(case)
+    try:
+        run.prefill()
+        run.decode_step(0)
+        st = run.cache.stats()
+        o = run.sim.snapshot()
+        np.testing.assert_array_equal(st["retained"].cpu().numpy(), o["n"])
+        np.testing.assert_array_equal(st["seen"].cpu().numpy(), o["pos"])
+        tot = st["totals"].cpu().numpy()
+        assert tot[0] == o["pos"].sum() and tot[1] == o["n"].sum()
+        for h in range(case.num_kv_heads):
+            ref = o["pos"][h::case.num_kv_heads].sum() / o["n"][h::case.num_kv_heads].sum()
+            assert abs(float(st["head_cr"][h]) - ref) <= 1e-6 * ref
+    finally:
+        run.close()
+
+
+def test_empty_and_partial_batches():
+    """Sequences never appended give zeros; decode over a subset, in any order."""
+    case = wl("subset", 5, 8, 2, 64, "bf16", 16, (0, 300), 3, 0.5, 23)
+    run = Run(case)
+    try:
+        run.prefill(seqs=[0, 2, 4])
+        ids = torch.tensor([1, 3], dtype=torch.int32, device="cuda")
+        q = torch.randn(2, 8, 64, device="cuda").to(torch.bfloat16)
+        out = run.cache.decode_attention(ids, q)
+        assert torch.count_nonzero(out) == 0
+        for step in range(3):
+            out, Q = run.decode_step(step, seqs=[4, 0])
+            torch.cuda.synchronize()
+            for k, b in enumerate([4, 0]):
+                compare(out[k], run.oracle_out(b, Q[k]))
+        run.check_metadata()
+    finally:
+        run.close()
+
+
+def test_f32_output_of_bf16_cache():
+    case = wl("outf32", 2, 8, 2, 128, "bf16", 16, (100, 400), 2, 0.5, 24)
+    run = Run(case)
+    try:
+        run.prefill()
+        for step in range(2):
+            out, Q = run.decode_step(step, out_dtype=torch.float32)
+            torch.cuda.synchronize()
+            assert out.dtype == torch.float32
+            for b in range(case.batch):
+                compare(out[b], run.oracle_out(b, Q[b]), max_abs=5e-3, mean_abs=5e-4)
+    finally:
+        run.close()
+
+
+def test_sequence_reset_returns_pages_in_order():
+    case = wl("reset", 3, 8, 2, 64, "bf16", 16, (50, 300), 2, 0.5, 25)
+    run = Run(case)
+    try:
+        run.prefill()
+        run.decode_step(0)
+        run.cache.reset_seq(1)
+        assert run.sim.reset_seq(1) == 0
+        run.seen[1] = 0
+        run._blk.pop(1, None)
+        run.check_metadata()
+        run.ctx[1] = 120
+        run.prefill(chunk=50, seqs=[1])
+        run.check_metadata()
+        out, Q = run.decode_step(1)
+        torch.cuda.synchronize()
+        for b in range(case.batch):
+            compare(out[b], run.oracle_out(b, Q[b]))
+        run.check_metadata()
+    finally:
+        run.close()
+
+
+def test_pool_exhaustion_latches_and_poisons():
+    case = wl("exhaust", 1, 4, 1, 64, "bf16", 16, (64, 64), 0, 0.0, 26)
+    run = Run(case, max_pages=4, check_sim=False)
+    try:
+        run.prefill()                   # 64 tokens, all kept: exactly 4 pages
+        assert run.cache.status() == _native.DMS_OK
+        run.decode_step(0)              # needs a 5th page
+        assert run.cache.status() == _native.DMS_ERR_POOL_EXHAUSTED
+        with pytest.raises(_native.DmsError) as e:
+            run.decode_step(1)
+        assert e.value.code == _native.DMS_ERR_POISONED
+        run.cache.reset()
+        assert run.cache.status() == _native.DMS_OK
+        snap = run.cache.snapshot()
+        assert snap["free_count"] == 4 and snap["n"].sum() == 0
+    finally:
+        run.close()
+
+
+def test_bulk_pool_exhaustion_and_bad_seq():
+    case = wl("bulk-exhaust", 2, 4, 1, 64, "bf16", 16, (100, 100), 0, 0.0, 27)
+    run = Run(case, max_pages=8, check_sim=False)
+    try:
+        run.prefill()                   # 2 x 100 tokens need 14 pages > 8
+        assert run.cache.status() == _native.DMS_ERR_POOL_EXHAUSTED
+        run.cache.reset()
+        ids = torch.tensor([5], dtype=torch.int32, device="cuda")   # max_seqs is 2
+        k = torch.zeros(1, 1, 64, dtype=torch.bfloat16, device="cuda")
+        run.cache.append(ids, k, k, torch.zeros(1, 1, dtype=torch.uint8, device="cuda"))
+        assert run.cache.status() == _native.DMS_ERR_BAD_SEQ
+    finally:
+        run.close()
+
+
+def test_host_argument_checks():
+    case = wl("args", 1, 4, 1, 64, "bf16", 16, (10, 10), 0, 0.5, 28)
+    run = Run(case, check_sim=False)
+    try:
+        ids = torch.tensor([0], dtype=torch.int32, device="cuda")
+        q = torch.zeros(1, 12, 64, dtype=torch.bfloat16, device="cuda")   # g = 12 > 8
+        with pytest.raises(_native.DmsError) as e:
+            run.cache.decode_attention(ids, q)
+        assert e.value.code == _native.DMS_ERR_INVALID
+        k = torch.zeros(2, 1, 64, dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(_native.DmsError):   # 2 rows for 1 sequence without cu_tokens
+            run.cache.append(ids, k, k, torch.zeros(2, 1, dtype=torch.uint8, device="cuda"))
+    finally:
+        run.close()
+    from learned_kv_cache_decode_b200 import DmsCache
+    for bad in (dict(head_dim=96), dict(window=0), dict(max_pages=0)):
+        args = dict(max_seqs=1, num_kv_heads=1, head_dim=64, window=4, max_pages=4, max_pages_per_stream=4)
+        args.update(bad)
+        with pytest.raises(_native.DmsError):
+            DmsCache(**args)
