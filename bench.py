@@ -1,0 +1,486 @@
+#!/usr/bin/env python
+"""Benchmark of the DMS decode step on B200: retained-KV HBM GB/s and decode steps/s.
+
+One step = for every layer cache: dms_append (one token per sequence, slot
+reuse, page pops), dms_stats, dms_decode_attention (split-K over the
+retained pages with the combine inside the same kernel). The prompt is
+bulk-appended beforehand (untimed). Inputs are seeded synthetic tensors with
+the shapes of the named workload (learned_kv_cache_decode_b200.workloads).
+
+Several layer caches with distinct pools are cycled inside every step so the
+retained K/V read per step is several times the 126 MB L2: timed reads come
+from HBM, not from L2.
+
+  python bench.py [--gpus N --steps K --warmup W --workload NAME --layers L]
+  python bench.py --impl reference ...   (the CPU oracle, timed on host cores)
+
+Under torchrun each rank runs its own replica on its own GPU (streams are
+independent; there is no data-path collective); rank 0 prints one JSON line
+with the whole-job value and the max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from learned_kv_cache_decode_b200 import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "retained-KV HBM GB/s and decode steps/sec (per layer, 1 B200) vs roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen-r1-7b-32k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--layers", type=int, default=0, help="layer caches per step (0: enough to exceed 8x L2)")
+    ap.add_argument("--attn-kernel", default="auto", choices=["auto", "mma", "simt"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# inputs
+
+def host_prompt(wl, seqs, ctx):
+    """Prompt K, V (bf16 bits or f32), alpha for the given sequences, concatenated in call order."""
+    Ks, Vs, As = [], [], []
+    for b, s in zip(seqs, ctx):
+        K, V = W.kv(wl, b, 0, int(s))
+        Ks.append(K)
+        Vs.append(V)
+        As.append(W.alpha(wl, b, 0, int(s)))
+    return np.concatenate(Ks), np.concatenate(Vs), np.concatenate(As)
+
+
+def host_decode(wl, seqs, ctx, steps):
+    """Decode-token inputs for `steps` steps: K, V [steps, B, Hkv, d], alpha [steps, B, Hkv], Q [steps, B, Hq, d]."""
+    Ks, Vs, As = [], [], []
+    for b, s in zip(seqs, ctx):
+        K, V = W.kv(wl, b, int(s), steps)
+        Ks.append(K)
+        Vs.append(V)
+        As.append(W.alpha(wl, b, int(s), steps))
+    K = np.stack(Ks, axis=1)
+    V = np.stack(Vs, axis=1)
+    A = np.stack(As, axis=1)
+    Q = np.stack([W.query(wl, 1_000_000 * (seqs[0] // wl.batch) + t)[[b % wl.batch for b in seqs]]
+                  for t in range(steps)])
+    return K, V, A, Q
+
+
+def to_torch(x, device):
+    import torch
+    if x.dtype == np.uint16:
+        t = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(x))
+    return t.to(device) if device is not None else t
+
+
+# ---------------------------------------------------------------------------
+# clocks (NVML reads only; nothing is changed)
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period: float = 0.005):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period = period
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml unavailable" if not self.ok else "no samples"}
+        names = [k for k, bit in self.REASONS.items() if self.reasons & bit and k != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples), "source": "nvml, 5 ms poll"}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(workload: str, kernel: str):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary,
+    valid only while the kernel source is unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", f"dms_decode_attention_{kernel}_{workload}.md")
+    src = os.path.join(ROOT, "learned_kv_cache_decode_b200", "csrc", "dms_attention.cu")
+    try:
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+        m_tr = re.search(r"traffic_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+        if m_sha and m_tr and m_sha.group(1) == sha:
+            return float(m_tr.group(1))
+    except OSError:
+        pass
+    return None
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle as it stands
+
+def oracle_sample(wl, seqs, steps_done, prompt, dec, n_items=None):
+    """Oracle inputs (float64) for the streams of `seqs` at their current last position."""
+    items, nbytes = [], 0
+    ctx = W.contexts(wl)
+    K_p, V_p, A_p, offs = prompt
+    Kd, Vd, Ad, Qd = dec
+    for k, b in enumerate(seqs):
+        s0, s1 = offs[k], offs[k + 1]
+        T = int(ctx[b % wl.batch]) + steps_done
+        Kfull = np.concatenate([K_p[s0:s1], Kd[:steps_done, k]])
+        Vfull = np.concatenate([V_p[s0:s1], Vd[:steps_done, k]])
+        Afull = np.concatenate([A_p[s0:s1], Ad[:steps_done, k]])
+        q = W.to_f64(Qd[max(steps_done - 1, 0), k])
+        g = wl.group
+        for h in range(wl.num_kv_heads):
+            a = Afull[:, h]
+            vis = int(np.count_nonzero((a == 0) | (np.arange(T) > T - 1 - wl.window)))
+            nbytes += vis * wl.head_dim * 2 * wl.elem_bytes
+            items.append((q[h * g:(h + 1) * g], W.to_f64(Kfull[:, h]), W.to_f64(Vfull[:, h]), a))
+            if n_items and len(items) >= n_items:
+                return items, nbytes
+    return items, nbytes
+
+
+def time_oracle(items, window, scale, target_s):
+    import oracle
+    reps, t_total, threads = 0, 0.0, 1
+    while t_total < target_s or reps == 0:
+        t0 = time.perf_counter()
+        _, threads = oracle.attention_batch(items, window, scale)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    return reps, t_total, threads
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    seqs = [0]
+    ctx = W.contexts(wl)[seqs]
+    K_p, V_p, A_p = host_prompt(wl, seqs, ctx)
+    offs = np.concatenate([[0], np.cumsum(ctx)])
+    dec = host_decode(wl, seqs, ctx, 1)
+    items, nbytes = oracle_sample(wl, seqs, 1, (K_p, V_p, A_p, offs), dec)
+    scale = 1.0 / math.sqrt(wl.head_dim)
+    import oracle
+    for _ in range(args.warmup):
+        oracle.attention_batch(items, wl.window, scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _, threads = oracle.attention_batch(items, wl.window, scale)
+    dt = time.perf_counter() - t0
+    value = nbytes * args.steps / dt / 1e9
+    sample = (f"{len(items)} streams (sequence 0, every KV head) of one decode step at the prompt's end; "
+              f"fp64 definition-form oracle, OpenMP over streams")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+def main():
+    args = parse_args()
+    wl = W.WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from learned_kv_cache_decode_b200 import DmsCache
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    # this rank's sequences (weak scaling: every rank runs a full batch of its own sequences)
+    seqs = [rank * wl.batch + b for b in range(wl.batch)]
+    ctx_all = W.contexts(wl)
+    ctx = np.array([ctx_all[b % wl.batch] for b in seqs])
+    B, hkv, hq, d = wl.batch, wl.num_kv_heads, wl.num_q_heads, wl.head_dim
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    n_dec = args.warmup + args.steps * (1 if args.no_e2e else 2)
+    mps = int((ctx.max() + n_dec) // 16 + 2)
+    scale = 1.0 / math.sqrt(d)
+
+    # prompt inputs (host, then device), shared by all layer caches
+    K_p, V_p, A_p = host_prompt(wl, seqs, ctx)
+    offs = np.concatenate([[0], np.cumsum(ctx)]).astype(np.int64)
+    dK, dV, dA = to_torch(K_p, dev), to_torch(V_p, dev), torch.from_numpy(A_p).to(dev)
+    d_cu = torch.from_numpy(offs.astype(np.int32)).to(dev)
+    ids = torch.arange(B, dtype=torch.int32, device=dev)   # cache-local sequence ids
+
+    def new_layer():
+        c = DmsCache(B, hkv, d, wl.window, B * hkv * mps, mps, dtype=tdt, attn_kernel=args.attn_kernel)
+        c.append(ids, dK, dV, dA, cu_tokens=d_cu)
+        return c
+
+    caches = [new_layer()]
+    torch.cuda.synchronize()
+    retained0 = int(caches[0].stats()["totals"][1])
+    layer_bytes = retained0 * d * 2 * wl.elem_bytes
+    L = args.layers or max(1, min(32, math.ceil(8 * L2_BYTES / max(layer_bytes, 1))))
+    caches += [new_layer() for _ in range(L - 1)]
+    torch.cuda.synchronize()
+    del dK, dV, dA
+    for c in caches:
+        if c.status() != 0:
+            raise RuntimeError(f"prefill failed: status {c.status()}")
+
+    # decode-step inputs: device-resident for the timed pass, pinned host for the e2e pass
+    Kd, Vd, Ad, Qd = host_decode(wl, seqs, ctx, n_dec)
+    t_K, t_V, t_A, t_Q = (to_torch(x, dev) for x in (Kd, Vd, Ad, Qd))
+    outs = [torch.empty((B, hq, d), dtype=tdt, device=dev) for _ in range(L)]
+    totals = torch.zeros((n_dec, L, 2), dtype=torch.int64, device=dev)
+
+    lib = caches[0].lib
+    hs = [c._h for c in caches]
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    row_kv = B * hkv * d * wl.elem_bytes
+    row_q = B * hq * d * wl.elem_bytes
+    pK, pV, pA, pQ = t_K.data_ptr(), t_V.data_ptr(), t_A.data_ptr(), t_Q.data_ptr()
+    pT = totals.data_ptr()
+    pids = ids.data_ptr()
+    launches0 = sum(c.launches() for c in caches)
+    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps * L)]
+
+    def step(t, timed):
+        for l in range(L):
+            h = hs[l]
+            rc = lib.dms_append(h, sp, B, pids, None, B, pK + t * row_kv, pV + t * row_kv, pA + t * B * hkv)
+            rc |= lib.dms_stats(h, sp, None, None, None, pT + (t * L + l) * 16)
+            if timed:
+                e0, e1 = ev_pairs[(t - args.warmup) * L + l]
+                e0.record(stream)
+            rc |= lib.dms_decode_attention(h, sp, B, pids, pQ + t * row_q, hq, scale, outs[l].data_ptr(),
+                                           0 if tdt == torch.bfloat16 else 1)
+            if timed:
+                e1.record(stream)
+            if rc:
+                raise RuntimeError(f"library call failed ({rc})")
+
+    for t in range(args.warmup):
+        step(t, False)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev_start, ev_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev_start.record(stream)
+        for t in range(args.warmup, args.warmup + args.steps):
+            step(t, True)
+        ev_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_ms = ev_start.elapsed_time(ev_end)
+    launches = sum(c.launches() for c in caches) - launches0
+    tot = totals.cpu().numpy()
+    timed_tot = tot[args.warmup:args.warmup + args.steps]           # [steps, L, 2]
+    bytes_launch = timed_tot[:, :, 1].astype(np.float64) * d * 2 * wl.elem_bytes
+    total_bytes = float(bytes_launch.sum())
+    attn_ms = np.array([a.elapsed_time(b) for a, b in ev_pairs])
+    status = [c.status() for c in caches]
+    if any(status):
+        raise RuntimeError(f"device status {status}")
+
+    # max over ranks of the timed region; whole-job bytes
+    t_max_ms, bytes_all = t_ms, total_bytes
+    if world > 1:
+        v = torch.tensor([t_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(v, op=dist.ReduceOp.MAX)
+        t_max_ms = float(v.item())
+        v = torch.tensor([total_bytes], dtype=torch.float64, device=dev)
+        dist.all_reduce(v, op=dist.ReduceOp.SUM)
+        bytes_all = float(v.item())
+    value = bytes_all / (t_max_ms * 1e-3) / 1e9
+
+    achieved = float(bytes_launch.mean()) / (float(attn_ms.mean()) * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+    kernel = {"auto": "mma" if tdt == torch.bfloat16 else "simt"}.get(args.attn_kernel, args.attn_kernel)
+
+    # ---- end-to-end pass through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hK, hV, hA, hQ = (to_torch(x, None).pin_memory() for x in (Kd, Vd, Ad, Qd))
+        h_out = [torch.empty((B, hq, d), dtype=tdt).pin_memory() for _ in range(L)]
+        stage = [(torch.empty((B, hkv, d), dtype=tdt, device=dev), torch.empty((B, hkv, d), dtype=tdt, device=dev),
+                  torch.empty((B, hkv), dtype=torch.uint8, device=dev), torch.empty((B, hq, d), dtype=tdt, device=dev))
+                 for _ in range(L)]
+        t0_e2e = args.warmup + args.steps
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_a.record(stream)
+        for t in range(t0_e2e, t0_e2e + args.steps):
+            for l in range(L):
+                k_, v_, a_, q_ = stage[l]
+                k_.copy_(hK[t], non_blocking=True)
+                v_.copy_(hV[t], non_blocking=True)
+                a_.copy_(hA[t], non_blocking=True)
+                q_.copy_(hQ[t], non_blocking=True)
+                caches[l].append(ids, k_, v_, a_)
+                lib.dms_stats(hs[l], sp, None, None, None, pT + (t * L + l) * 16)
+                caches[l].decode_attention(ids, q_, scale=scale, out=outs[l])
+                h_out[l].copy_(outs[l], non_blocking=True)
+        e_b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e_a.elapsed_time(e_b)
+        tot2 = totals.cpu().numpy()[t0_e2e:t0_e2e + args.steps]
+        e2e_bytes = float(tot2[:, :, 1].astype(np.float64).sum()) * d * 2 * wl.elem_bytes
+        if world > 1:
+            v = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(v, op=dist.ReduceOp.MAX)
+            e2e_ms = float(v.item())
+            v = torch.tensor([e2e_bytes], dtype=torch.float64, device=dev)
+            dist.all_reduce(v, op=dist.ReduceOp.SUM)
+            e2e_bytes = float(v.item())
+        h2d = L * (2 * row_kv + B * hkv + row_q)
+        d2h = L * B * hq * d * wl.elem_bytes
+        e2e = {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
+
+    # ---- CPU baseline: the oracle on a bounded sample of the same step (rank 0, N = 1)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample_seqs = list(range(min(B, 2)))
+        items, nbytes = oracle_sample(wl, [seqs[i] for i in sample_seqs], args.warmup + args.steps,
+                                      (K_p, V_p, A_p, offs),
+                                      (Kd[:, sample_seqs], Vd[:, sample_seqs], Ad[:, sample_seqs],
+                                       Qd[:, sample_seqs]))
+        reps, t_cpu, threads = time_oracle(items, wl.window, scale, args.cpu_seconds)
+        cpu = {"value": nbytes * reps / t_cpu / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{len(items)} streams (sequences {sample_seqs}, every KV head) at the last timed step, "
+                         f"repeated {reps}x ({t_cpu:.1f} s); fp64 definition-form oracle, OpenMP over streams"}
+
+    if rank == 0:
+        n_layer_steps = args.steps * L
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_max_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": {
+                "workload": wl.name, "batch_per_gpu": B, "q_heads": hq, "kv_heads": hkv, "head_dim": d,
+                "window": wl.window, "context": int(ctx.max()) if wl.ctx_range is None else list(wl.ctx_range),
+                "layers": L, "attn_kernel": kernel, "parallelism": f"replicas x{world}",
+                "l2": f"inputs larger than L2: {L} layer pools, {layer_bytes / 2**20:.0f} MiB retained K/V each "
+                      f"({L * layer_bytes / 2**20:.0f} MiB per step vs 126 MiB L2)",
+                "step": "per layer: dms_append (1 token/seq) + dms_stats + dms_decode_attention",
+            },
+            "decode_steps_per_s_per_layer": n_layer_steps / (t_max_ms * 1e-3),
+            "retained_bytes_per_step": total_bytes / args.steps,
+            "compression_ratio": float(timed_tot[-1, :, 0].sum() / timed_tot[-1, :, 1].sum()),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "traffic": profile_traffic(wl.name, kernel),
+                         "kernel": f"dms_decode_attention ({kernel})",
+                         "launch_ms_mean": float(attn_ms.mean()), "launch_ms_p10": float(np.percentile(attn_ms, 10)),
+                         "launch_ms_p90": float(np.percentile(attn_ms, 90)),
+                         "bytes_per_launch": float(bytes_launch.mean())},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+
+    for c in caches:
+        c.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
