@@ -103,9 +103,10 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
   step(alloc(&dv.scratch, S));
   step(alloc(&dv.cnt, S));
   step(alloc(&dv.kv, (size_t)dv.max_pages * 2 * dms::kPage * dv.d * dv.elem_bytes));
+  if (e == cudaSuccess) e = dms::prepare_aux_kernels();
   if (e == cudaSuccess) e = dms::attention_prepare(dv, c.dtype, c.attn_kernel, h->num_sms, &h->plan);
   if (e == cudaSuccess)
-    e = alloc(&dv.part, (size_t)(h->plan.grid + dv.S) * dms::kMaxGroup * (dv.d + 2));
+    e = alloc(&dv.part, ((size_t)h->plan.grid + dv.S) * dms::kMaxGroup * (dv.d + 2));
   if (e == cudaSuccess) e = cudaMemset(dv.kv, 0, (size_t)dv.max_pages * 2 * dms::kPage * dv.d * dv.elem_bytes);
   if (e == cudaSuccess) e = cudaMemset(dv.page_table, 0xff, S * dv.mps * sizeof(int32_t));
   if (e == cudaSuccess) e = cudaMemset(dv.slot_pos, 0xff, (size_t)dv.max_pages * dms::kPage * sizeof(int32_t));

@@ -419,6 +419,22 @@ gather_kernel(Dev dv, int seq, int kvh, int rows_cap, uint8_t* Kout, uint8_t* Vo
 
 // ---------------------------------------------------------------------------
 
+// The attention kernel runs with nearly all of shared memory; giving every
+// bookkeeping kernel the same carveout preference spares the SMs a
+// reconfiguration between consecutive launches.
+cudaError_t prepare_aux_kernels() {
+  const void* fns[] = {(const void*)append_decode_kernel, (const void*)bulk_count_kernel,
+                       (const void*)bulk_pages_kernel, (const void*)bulk_write_kernel,
+                       (const void*)reset_seq_kernel, (const void*)init_state_kernel,
+                       (const void*)stats_kernel, (const void*)gather_kernel};
+  for (const void* f : fns) {
+    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_init_state(const Dev& dv, cudaStream_t st) {
   init_state_kernel<<<256, 256, 0, st>>>(dv);
   return cudaGetLastError();

@@ -32,6 +32,8 @@
 //    section 3.2 "Performance Considerations").
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
+#include <cstdlib>
 #include <type_traits>
 
 #include "dms_internal.cuh"
@@ -54,6 +56,8 @@ struct AttnArgs {
   int32_t* cnt;
   int n_seqs, hkv, g, hq, mps, max_seqs, max_pages, out_f32;
   float sl2e;   // softmax scale * log2(e): scores live in the base-2 domain
+  int spw;      // TMA stages per warp
+  int S;        // streams of the cache (sizes the plan arrays in shared memory)
 };
 
 // Largest i in [0, n] with prefix[i] <= x (prefix is non-decreasing, prefix[0] = 0).
@@ -66,15 +70,18 @@ __device__ __forceinline__ int stream_of(const int* prefix, int n, int x) {
   return lo;
 }
 
-// CTA that owns global page index x when P pages are cut into G ranges
-// [floor(c P / G), floor((c+1) P / G)).
-__device__ __forceinline__ int cta_of(long long x, long long P, long long G) {
+// Range (CTA) that owns global page index x when P pages are cut into G
+// ranges [floor(c P / G), floor((c+1) P / G)), all of them non-empty (G <= P).
+__device__ __forceinline__ int range_of(long long x, long long P, long long G) {
   return (int)(((x + 1) * G - 1) / P);
 }
 
+// Partial result of one (CTA range, stream) piece: unnormalised output
+// O[head][d], running max m[head] (base-2 domain) and sum l[head]. The same
+// layout serves as a warp's slot in the CTA merge area in shared memory.
 template <int D>
-struct MergeSmem {   // one slot per consumer warp
-  float acc[kMaxGroup][D];
+struct Partial {
+  float O[kMaxGroup][D];
   float m[kMaxGroup];
   float l[kMaxGroup];
 };
@@ -116,71 +123,118 @@ __device__ __forceinline__ uint32_t sw128(uint32_t stage, int row, int chunk) {
   return stage + (uint32_t)((chunk >> 3) * 4096 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
+// Per-lane byte offsets (within a stage) of the ldmatrix rows this lane
+// addresses: K tiles for QK (rows 0..15) and V tiles for PV (rows 16..31).
 template <int D>
-__device__ __forceinline__ void mma_page(MmaState<D>& S, uint32_t stage, int valid, float sl2e, int lane) {
-  // ---- S^T = K * Q^T : rows = 16 tokens, cols = 8 heads
-  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-  const int krow = lane & 15;
+struct MmaOffsets {
+  uint32_t k[D / 16], v[D / 16];
+  __device__ __forceinline__ explicit MmaOffsets(int lane) {
+    const int krow = lane & 15;
+    const int vrow = 16 + ((lane >> 4) << 3) + (lane & 7);
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    uint32_t af[4];
-    ldsm_x4(sw128(stage, krow, 2 * kk + (lane >> 4)), af);
-    if (kk & 1) mma_16816(sb, af, S.qb[kk][0], S.qb[kk][1]);
-    else        mma_16816(sa, af, S.qb[kk][0], S.qb[kk][1]);
+    for (int t = 0; t < D / 16; ++t) {
+      k[t] = sw128(0, krow, 2 * t + (lane >> 4));
+      v[t] = sw128(0, vrow, 2 * t + ((lane >> 3) & 1));
+    }
   }
-  float v0 = (sa[0] + sb[0]) * sl2e, v1 = (sa[1] + sb[1]) * sl2e;   // token t0 = lane/4
-  float v2 = (sa[2] + sb[2]) * sl2e, v3 = (sa[3] + sb[3]) * sl2e;   // token t0 + 8
+};
+
+// NP pages of one stream at once: their QK products, one shared online-
+// softmax update, then their PV products. `valid[p]` tokens of page p are
+// real (16 except in a stream's last page).
+template <int D, int NP>
+__device__ __forceinline__ void mma_pages(MmaState<D>& S, const uint32_t (&stage)[NP], const int (&valid)[NP],
+                                          float sl2e, int lane, const MmaOffsets<D>& off) {
+  // ---- S^T = K * Q^T per page: rows = 16 tokens, cols = 8 heads
+  float v[NP][4];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t af[4];
+      ldsm_x4(stage[p] + off.k[kk], af);
+      if (kk & 1) mma_16816(sb, af, S.qb[kk][0], S.qb[kk][1]);
+      else        mma_16816(sa, af, S.qb[kk][0], S.qb[kk][1]);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) v[p][r] = (sa[r] + sb[r]) * sl2e;   // r 0,1: token lane/4; 2,3: +8
+  }
   const int t0 = lane >> 2;
-  if (valid < kPage) {
-    if (t0 >= valid)     { v0 = -INFINITY; v1 = -INFINITY; }
-    if (t0 + 8 >= valid) { v2 = -INFINITY; v3 = -INFINITY; }
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    if (valid[p] < kPage) {
+      if (t0 >= valid[p])     { v[p][0] = -INFINITY; v[p][1] = -INFINITY; }
+      if (t0 + 8 >= valid[p]) { v[p][2] = -INFINITY; v[p][3] = -INFINITY; }
+    }
   }
   // ---- online softmax per head column (tokens spread over lanes with equal lane % 4)
-  float mx0 = fmaxf(v0, v2), mx1 = fmaxf(v1, v3);
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    mx0 = fmaxf(mx0, fmaxf(v[p][0], v[p][2]));
+    mx1 = fmaxf(mx1, fmaxf(v[p][1], v[p][3]));
+  }
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
   }
   const float mn0 = fmaxf(S.m[0], mx0), mn1 = fmaxf(S.m[1], mx1);
-  const float c0 = ex2(S.m[0] - mn0), c1 = ex2(S.m[1] - mn1);
-  const float p0 = ex2(v0 - mn0), p1 = ex2(v1 - mn1);
-  const float p2 = ex2(v2 - mn0), p3 = ex2(v3 - mn1);
-  S.m[0] = mn0;
-  S.m[1] = mn1;
-  S.l[0] = S.l[0] * c0 + p0 + p2;
-  S.l[1] = S.l[1] * c1 + p1 + p3;
+  float pr[NP][4];
+  float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-  for (int mt = 0; mt < D / 16; ++mt) {
-    S.acc[mt][0] *= c0;
-    S.acc[mt][1] *= c1;
-    S.acc[mt][2] *= c0;
-    S.acc[mt][3] *= c1;
+  for (int p = 0; p < NP; ++p) {
+    pr[p][0] = ex2(v[p][0] - mn0);
+    pr[p][1] = ex2(v[p][1] - mn1);
+    pr[p][2] = ex2(v[p][2] - mn0);
+    pr[p][3] = ex2(v[p][3] - mn1);
+    sum0 += pr[p][0] + pr[p][2];
+    sum1 += pr[p][1] + pr[p][3];
   }
-  // ---- P^T as B fragments: transpose the [token][head] C fragments
-  const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));   // tokens 0..7
-  const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));   // tokens 8..15
-  // ---- O^T += V^T * P^T : rows = head_dim (16 per tile), cols = heads
-  const int vrow = 16 + ((lane >> 4) << 3) + (lane & 7);
+  if (__any_sync(0xffffffffu, (mn0 != S.m[0]) | (mn1 != S.m[1]))) {   // the running max moved
+    const float c0 = ex2(S.m[0] - mn0), c1 = ex2(S.m[1] - mn1);
+    S.l[0] *= c0;
+    S.l[1] *= c1;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      S.acc[mt][0] *= c0;
+      S.acc[mt][1] *= c1;
+      S.acc[mt][2] *= c0;
+      S.acc[mt][3] *= c1;
+    }
+    S.m[0] = mn0;
+    S.m[1] = mn1;
+  }
+  S.l[0] += sum0;
+  S.l[1] += sum1;
+  // ---- O^T += V^T * P^T per page: rows = head_dim (16 per tile), cols = heads
   const int tk = 2 * (lane & 3);   // tokens of this lane in a0/a1 (and +8 in a2/a3)
 #pragma unroll
-  for (int mt = 0; mt < D / 16; ++mt) {
-    uint32_t af[4];
-    ldsm_x4_trans(sw128(stage, vrow, 2 * mt + ((lane >> 3) & 1)), af);
-    if (valid < kPage) {   // rows past n may hold stale bits: zero them
-      const uint32_t lo0 = tk < valid ? 0x0000ffffu : 0u, hi0 = tk + 1 < valid ? 0xffff0000u : 0u;
-      const uint32_t lo1 = tk + 8 < valid ? 0x0000ffffu : 0u, hi1 = tk + 9 < valid ? 0xffff0000u : 0u;
-      af[0] &= lo0 | hi0;
-      af[1] &= lo0 | hi0;
-      af[2] &= lo1 | hi1;
-      af[3] &= lo1 | hi1;
+  for (int p = 0; p < NP; ++p) {
+    const uint32_t pb0 = movmatrix_trans(pack_bf16x2(pr[p][0], pr[p][1]));   // tokens 0..7
+    const uint32_t pb1 = movmatrix_trans(pack_bf16x2(pr[p][2], pr[p][3]));   // tokens 8..15
+    uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
+    if (valid[p] < kPage) {   // rows past n may hold stale bits: zero them
+      keep0 = (tk < valid[p] ? 0x0000ffffu : 0u) | (tk + 1 < valid[p] ? 0xffff0000u : 0u);
+      keep1 = (tk + 8 < valid[p] ? 0x0000ffffu : 0u) | (tk + 9 < valid[p] ? 0xffff0000u : 0u);
     }
-    mma_16816(S.acc[mt], af, pb0, pb1);
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      uint32_t af[4];
+      ldsm_x4_trans(stage[p] + off.v[mt], af);
+      af[0] &= keep0;
+      af[1] &= keep0;
+      af[2] &= keep1;
+      af[3] &= keep1;
+      mma_16816(S.acc[mt], af, pb0, pb1);
+    }
   }
 }
 
+// Write a warp's tensor-core state (fragments) into its merge slot.
 template <int D>
-__device__ __forceinline__ void mma_to_smem(MmaState<D>& S, MergeSmem<D>* slot, int lane) {
+__device__ __forceinline__ void mma_to_slot(const MmaState<D>& S, Partial<D>* slot, int lane) {
   float l0 = S.l[0], l1 = S.l[1];
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
@@ -190,10 +244,10 @@ __device__ __forceinline__ void mma_to_smem(MmaState<D>& S, MergeSmem<D>* slot, 
   const int h0 = 2 * (lane & 3), r0 = lane >> 2;
 #pragma unroll
   for (int mt = 0; mt < D / 16; ++mt) {
-    slot->acc[h0][mt * 16 + r0] = S.acc[mt][0];
-    slot->acc[h0 + 1][mt * 16 + r0] = S.acc[mt][1];
-    slot->acc[h0][mt * 16 + r0 + 8] = S.acc[mt][2];
-    slot->acc[h0 + 1][mt * 16 + r0 + 8] = S.acc[mt][3];
+    slot->O[h0][mt * 16 + r0] = S.acc[mt][0];
+    slot->O[h0 + 1][mt * 16 + r0] = S.acc[mt][1];
+    slot->O[h0][mt * 16 + r0 + 8] = S.acc[mt][2];
+    slot->O[h0 + 1][mt * 16 + r0 + 8] = S.acc[mt][3];
   }
   if (r0 == 0) {
     slot->m[h0] = S.m[0];
@@ -268,11 +322,11 @@ __device__ __forceinline__ void simt_page(SimtState<D>& S, const E* stage, int v
 }
 
 template <int D>
-__device__ __forceinline__ void simt_to_smem(SimtState<D>& S, MergeSmem<D>* slot, int lane) {
+__device__ __forceinline__ void simt_to_slot(const SimtState<D>& S, Partial<D>* slot, int lane) {
 #pragma unroll
   for (int h = 0; h < kMaxGroup; ++h) {
 #pragma unroll
-    for (int e = 0; e < D / 32; ++e) slot->acc[h][lane * (D / 32) + e] = S.acc[h][e];
+    for (int e = 0; e < D / 32; ++e) slot->O[h][lane * (D / 32) + e] = S.acc[h][e];
     if (lane == 0) {
       slot->m[h] = S.m[h];
       slot->l[h] = S.l[h];
@@ -292,29 +346,47 @@ __device__ __forceinline__ void store_out(const AttnArgs& a, int b, int h, int d
   }
 }
 
-// Stage ring. Page c of a CTA goes to consumer warp c % NCW, which owns SPW
-// private stages and uses them in order: every stage's mbarrier phases are
-// then waited on by exactly one warp, one phase after the other, so a
-// parity wait can never match a phase two steps old.
-template <int NCW, int SPW>
-__device__ __forceinline__ int stage_of(int c) { return (c % NCW) * SPW + (c / NCW) % SPW; }
-template <int NCW, int SPW>
-__device__ __forceinline__ int phase_of(int c) { return (c / NCW) / SPW; }
+// Shared-memory layout of one CTA (byte offsets from a 1024-aligned base).
+struct SmemLayout {
+  int stages, bars, misc, merge, prefix, sid, total;
+};
 
-template <int D, int NCW, int SPW, bool MMA, typename E>
-__global__ void __launch_bounds__((NCW + 1) * 32, 1)
+__host__ __device__ inline SmemLayout smem_layout(int ncw, int spw, int stage_bytes, int d, int S) {
+  SmemLayout L;
+  L.stages = 0;
+  L.bars = ncw * spw * stage_bytes;
+  L.misc = L.bars + 8 * ncw * spw;
+  L.merge = L.misc + 64;
+  L.prefix = L.merge + ncw * kMaxGroup * (d + 2) * 4;
+  L.sid = L.prefix + (S + 1) * 4;
+  L.total = L.sid + S * 4;
+  return L;
+}
+
+// Split-K over CTA ranges. The call's retained pages, stream after stream,
+// are cut into gridDim.x equal contiguous ranges, one per CTA. Page c of a
+// range goes to warp c % NCW, which runs its own TMA pipeline over `spw`
+// private stages: it refills a stage as soon as it has computed on it, and
+// every stage's mbarrier phases are waited on by that one warp, in order.
+// At the end of each stream piece the warps' softmax states are merged in
+// shared memory; a split stream leaves one partial per CTA and the last CTA
+// to finish it combines them (a few partials per stream). The next piece's
+// query is loaded before the merge, and the copies already in flight keep
+// HBM busy while the CTA merges.
+template <int D, int NCW, int NB, bool MMA, typename E>
+__global__ void __launch_bounds__(NCW * 32, 1)
 attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
-  constexpr int NSTAGES = NCW * SPW;
-  constexpr int kThreads = (NCW + 1) * 32;
+  constexpr int kThreads = NCW * 32;
   constexpr int kStage = 2 * kPage * D * (int)sizeof(E);   // one page: 16 K rows + 16 V rows
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* stages = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + NSTAGES * kStage);
-  uint64_t* empty = full + NSTAGES;
-  int* misc = reinterpret_cast<int*>(empty + NSTAGES);   // [0] abort, [1] ok, [2] last, [3..10] scan
-  MergeSmem<D>* mrg = reinterpret_cast<MergeSmem<D>*>(misc + 16);
-  int* prefix = reinterpret_cast<int*>(mrg + NCW);
+  const int spw = a.spw;
+  const SmemLayout lay = smem_layout(NCW, spw, kStage, D, a.S);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
+  int* misc = reinterpret_cast<int*>(smem + lay.misc);   // [0] abort, [1] ok, [2] last, [3..] scan scratch
+  Partial<D>* slots = reinterpret_cast<Partial<D>*>(smem + lay.merge);
+  int* prefix = reinterpret_cast<int*>(smem + lay.prefix);
+  int* sid = reinterpret_cast<int*>(smem + lay.sid);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nst = a.n_seqs * a.hkv;
@@ -323,28 +395,27 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   if (tid == 0) {
     misc[0] = 0;
     misc[1] = (read_status(a.ctrl) == 0);
-    for (int s = 0; s < NSTAGES; ++s) {
-      mbar_init(smem_addr(&full[s]), 1);
-      mbar_init(smem_addr(&empty[s]), 1);
-    }
+    for (int s = 0; s < NCW * spw; ++s) mbar_init(smem_addr(&full[s]), 1);
     fence_mbar_init();
   }
   __syncthreads();
   if (!misc[1]) return;   // poisoned cache: do nothing
 
-  // ---- plan: retained pages per stream of the call, prefix in smem
+  // ---- plan: retained pages per stream of the call (prefix) and stream ids, in smem
   {
     const int per = (nst + kThreads - 1) / kThreads;
     const int b0 = min(tid * per, nst), e0 = min(b0 + per, nst);
     int local = 0;
     for (int i = b0; i < e0; ++i) {
       const int seq = a.seq_ids[i / a.hkv];
-      int pages = 0;
+      int pages = 0, st = 0;
       if (seq < 0 || seq >= a.max_seqs) {
         latch(a.ctrl, DMS_ERR_BAD_SEQ);
       } else {
-        pages = (a.n[seq * a.hkv + i % a.hkv] + kPage - 1) / kPage;
+        st = seq * a.hkv + i % a.hkv;
+        pages = (a.n[st] + kPage - 1) / kPage;
       }
+      sid[i] = st;
       prefix[i + 1] = pages;
       local += pages;
     }
@@ -367,154 +438,174 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     for (int e = tid; e < a.g * D; e += kThreads) store_out(a, b, kvh * a.g + e / D, e % D, D, 0.f);
   }
   const long long Geff = P < G ? P : G;
-  if (blockIdx.x >= Geff) return;
-  const int K0 = (int)(blockIdx.x * P / Geff);
-  const int K1 = (int)((blockIdx.x + 1) * P / Geff);
+  if (blockIdx.x >= Geff) return;   // uniform over the CTA
+  const int K0 = (int)(blockIdx.x * P / Geff), K1 = (int)((blockIdx.x + 1) * P / Geff);
   const int ncta = K1 - K0;
 
-  if (warp == NCW) {
-    // ================= producer warp =================
-    const int bytes_per_row = D * (int)sizeof(E);
-    auto lookup = [&](int c) -> int {
-      if (c >= ncta) return -1;
-      const int kk = K0 + c;
-      const int i = stream_of(prefix, nst, kk);
-      const int p = kk - prefix[i];
-      const int st = a.seq_ids[i / a.hkv] * a.hkv + i % a.hkv;
-      int pg = __ldg(a.page_table + (size_t)st * a.mps + p);
-      if (pg < 0 || pg >= a.max_pages) {
-        latch(a.ctrl, DMS_ERR_INVALID);
-        pg = 0;
-      }
-      return pg;
-    };
-    int issued = 0;   // lane 0: pages whose copy was issued (in order)
-    int pg_next = lookup(lane);
-    for (int base = 0; base < ncta; base += 32) {
-      const int pg_cur = pg_next;
-      pg_next = lookup(base + 32 + lane);   // next batch, overlapped with this one
-      const int nb = min(32, ncta - base);
-      for (int j = 0; j < nb; ++j) {
-        const int pg = __shfl_sync(0xffffffffu, pg_cur, j);
-        if (lane == 0 && !*abort_flag) {
-          const int c = base + j;
-          const int s = stage_of<NCW, SPW>(c), ph = phase_of<NCW, SPW>(c);
-          bool go = true;
-          if (ph > 0) go = mbar_wait_bounded(smem_addr(&empty[s]), (ph - 1) & 1, abort_flag, a.ctrl);
-          if (go) {
-            const uint32_t dst = smem_addr(stages + s * kStage);
-            const uint32_t bar = smem_addr(&full[s]);
-            mbar_arrive_expect_tx(bar, kStage);
-            if constexpr (MMA) {
-#pragma unroll
-              for (int box = 0; box < D / 64; ++box) tma_load_3d(dst + box * 4096, &tmap, bar, box * 64, 0, pg);
-            } else {
-              bulk_load(dst, a.kv + (size_t)pg * 2 * kPage * bytes_per_row, kStage, bar);
-            }
-            issued = c + 1;
-          }
-        }
-        __syncwarp();
-      }
+  // ---- this warp's page pipeline: CTA pages c = warp + NCW * j, j = 0 .. njobs-1
+  const int njobs = ncta > warp ? (ncta - warp + NCW - 1) / NCW : 0;
+  uint64_t* myfull = full + warp * spw;
+  uint8_t* mystage = smem + lay.stages + (size_t)warp * spw * kStage;
+  auto lookup = [&](int j) -> int {   // physical page of the warp's j-th page
+    if (j >= njobs) return 0;
+    const int kk = K0 + warp + NCW * j;
+    const int i = stream_of(prefix, nst, kk);
+    int pg = __ldg(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i]));
+    if (pg < 0 || pg >= a.max_pages) {
+      latch(a.ctrl, DMS_ERR_INVALID);
+      pg = 0;
     }
-    // Drain: every issued copy must land before the CTA can exit (bounded).
-    // The last NSTAGES issued pages use distinct stages.
+    return pg;
+  };
+  int jb = 0;                                     // page ids of jobs [jb, jb+32) in pid_cur,
+  int pid_cur = lookup(lane), pid_nxt = lookup(32 + lane);   // [jb+32, jb+64) in pid_nxt
+  int issued = 0;
+  auto issue = [&](int j) {   // warp-uniform; j = issued
+    if (j - jb >= 32) {
+      pid_cur = pid_nxt;
+      jb += 32;
+      pid_nxt = lookup(jb + 32 + lane);
+    }
+    const int r = j - jb;
+    const int pg = __shfl_sync(0xffffffffu, r < 32 ? pid_cur : pid_nxt, r & 31);
     if (lane == 0) {
-      for (int c = max(0, issued - NSTAGES); c < issued; ++c)
-        mbar_wait_timed(smem_addr(&full[stage_of<NCW, SPW>(c)]), phase_of<NCW, SPW>(c) & 1, a.ctrl);
+      const int s = j % spw;
+      const uint32_t bar = smem_addr(&myfull[s]);
+      const uint32_t dst = smem_addr(mystage + (size_t)s * kStage);
+      mbar_arrive_expect_tx(bar, kStage);
+      if constexpr (MMA) {
+#pragma unroll
+        for (int box = 0; box < D / 64; ++box) tma_load_3d(dst + box * 4096, &tmap, bar, box * 64, 0, pg);
+      } else {
+        bulk_load(dst, a.kv + (size_t)pg * kStage, kStage, bar);
+      }
     }
-    return;
-  }
+    issued = j + 1;
+  };
+  for (int j = 0; j < spw && j < njobs; ++j) issue(j);
 
-  // ================= consumer warps =================
   using State = typename std::conditional<MMA, MmaState<D>, SimtState<D>>::type;
   State S;
+  const MmaOffsets<D> off(lane);
+  int consumed = 0;
   int k = K0;
+  int i = stream_of(prefix, nst, k);
+  if constexpr (MMA) mma_load_q<D>(S, a, i / a.hkv, i % a.hkv, lane);
+  else simt_load_q<D, E>(S, a, i / a.hkv, i % a.hkv, lane);
+  int nn = __ldg(a.n + sid[i]);
   while (k < K1) {
-    const int i = stream_of(prefix, nst, k);
     const int pstart = prefix[i], pend = prefix[i + 1];
-    const int pb = k, pe = min(pend, K1);
+    const int pe = min(pend, K1);
     const int b = i / a.hkv, kvh = i % a.hkv;
-    const int st = a.seq_ids[b] * a.hkv + kvh;
-    const int nn = __ldg(a.n + st);
-    const bool whole = (pb == pstart) && (pe == pend);
-    if constexpr (MMA) mma_load_q<D>(S, a, b, kvh, lane);
-    else simt_load_q<D, E>(S, a, b, kvh, lane);
+    const bool whole = (k == pstart) && (pe == pend);
 
-    const int rel = pb - K0;
-    const int c_first = rel + ((warp - rel) % NCW + NCW) % NCW;
-    for (int c = c_first; c < pe - K0; c += NCW) {
-      const int s = stage_of<NCW, SPW>(c);
-      const bool ok = mbar_wait_bounded(smem_addr(&full[s]), phase_of<NCW, SPW>(c) & 1, abort_flag, a.ctrl);
+    const int rel = k - K0;
+    for (int c = rel + ((warp - rel) % NCW + NCW) % NCW; c < pe - K0;) {
+      const int j = (c - warp) / NCW;
+      const int nb = (NB == 2 && c + NCW < pe - K0) ? 2 : 1;   // pages in this batch (same stream)
+      bool ok = mbar_wait_bounded(smem_addr(&myfull[j % spw]), (j / spw) & 1, abort_flag, a.ctrl);
+      if (nb == 2) ok &= mbar_wait_bounded(smem_addr(&myfull[(j + 1) % spw]), ((j + 1) / spw) & 1, abort_flag, a.ctrl);
       if (ok) {
-        const int p = K0 + c - pstart;
-        const int valid = (K0 + c == pend - 1) ? nn - kPage * p : kPage;
-        if constexpr (MMA) mma_page<D>(S, smem_addr(stages + s * kStage), valid, a.sl2e, lane);
-        else simt_page<D, E>(S, reinterpret_cast<const E*>(stages + s * kStage), valid, a.g, lane);
+        const int p = K0 + c - pstart;   // page index within the stream
+        const int valid0 = (K0 + c == pend - 1) ? nn - kPage * p : kPage;
+        const uint8_t* st0 = mystage + (size_t)(j % spw) * kStage;
+        if constexpr (MMA) {
+          if (nb == 2) {
+            const int valid1 = (K0 + c + NCW == pend - 1) ? nn - kPage * (p + NCW) : kPage;
+            const uint32_t stg[2] = {smem_addr(st0), smem_addr(mystage + (size_t)((j + 1) % spw) * kStage)};
+            const int val[2] = {valid0, valid1};
+            mma_pages<D, 2>(S, stg, val, a.sl2e, lane, off);
+          } else {
+            const uint32_t stg[1] = {smem_addr(st0)};
+            const int val[1] = {valid0};
+            mma_pages<D, 1>(S, stg, val, a.sl2e, lane, off);
+          }
+        } else {
+          simt_page<D, E>(S, reinterpret_cast<const E*>(st0), valid0, a.g, lane);
+        }
       }
+      consumed = j + nb;
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&empty[s]));
+      const bool stop = __any_sync(0xffffffffu, *abort_flag != 0);
+      for (int q = 0; q < nb; ++q)
+        if (j + q + spw < njobs && !stop) issue(j + q + spw);
+      c += nb * NCW;
     }
 
-    // ---- merge the warps' states for this piece
-    if constexpr (MMA) mma_to_smem<D>(S, &mrg[warp], lane);
-    else simt_to_smem<D>(S, &mrg[warp], lane);
-    named_barrier(1, NCW * 32);
+    // ---- end of the piece: merge the warps' states in shared memory
+    if constexpr (MMA) mma_to_slot<D>(S, &slots[warp], lane);
+    else simt_to_slot<D>(S, &slots[warp], lane);
+    // start loading the next piece's query while the CTA merges
+    const int inext = pe < K1 ? stream_of(prefix, nst, pe) : i;
+    if (pe < K1) {
+      if constexpr (MMA) mma_load_q<D>(S, a, inext / a.hkv, inext % a.hkv, lane);
+      else simt_load_q<D, E>(S, a, inext / a.hkv, inext % a.hkv, lane);
+    }
+    const int nn_next = pe < K1 ? __ldg(a.n + sid[inext]) : 0;
+    __syncthreads();
 
-    const int slot = blockIdx.x + i;   // partial slot of piece (CTA, stream)
-    float* part = a.part + (size_t)slot * kMaxGroup * (D + 2);
-    for (int e = tid; e < a.g * D; e += NCW * 32) {
+    Partial<D>* part = reinterpret_cast<Partial<D>*>(a.part) + (blockIdx.x + i);
+    for (int e = tid; e < a.g * D; e += kThreads) {
       const int h = e / D, dd = e % D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < NCW; ++w) M = fmaxf(M, mrg[w].m[h]);
+      for (int w = 0; w < NCW; ++w) M = fmaxf(M, slots[w].m[h]);
       float L = 0.f, O = 0.f;
 #pragma unroll
       for (int w = 0; w < NCW; ++w) {
-        const float mw = mrg[w].m[h];
+        const float mw = slots[w].m[h];
         if (mw == -INFINITY) continue;
         const float sc = ex2(mw - M);
-        L += mrg[w].l[h] * sc;
-        O += mrg[w].acc[h][dd] * sc;
+        L += slots[w].l[h] * sc;
+        O += slots[w].O[h][dd] * sc;
       }
       if (whole) {
         store_out(a, b, kvh * a.g + h, dd, D, O / L);
       } else {
-        part[h * D + dd] = O;
+        part->O[h][dd] = O;
         if (dd == 0) {
-          part[kMaxGroup * D + h] = M;
-          part[kMaxGroup * D + kMaxGroup + h] = L;
+          part->m[h] = M;
+          part->l[h] = L;
         }
       }
     }
     if (!whole) {
-      __threadfence();
-      named_barrier(1, NCW * 32);
-      const int first = cta_of(pstart, P, Geff), last = cta_of(pend - 1, P, Geff);
-      if (tid == 0) misc[2] = (atomicAdd(&a.cnt[i], 1) == last - first);
-      named_barrier(1, NCW * 32);
-      if (misc[2]) {
-        __threadfence();
-        for (int e = tid; e < a.g * D; e += NCW * 32) {
+      __syncthreads();   // the partial is complete in this CTA ...
+      const int first = range_of(pstart, P, Geff), last = range_of(pend - 1, P, Geff);
+      if (tid == 0) {
+        __threadfence();   // ... and visible device-wide before the count moves
+        misc[2] = (atomicAdd(&a.cnt[i], 1) == last - first);
+        if (misc[2]) __threadfence();
+      }
+      __syncthreads();
+      if (misc[2]) {   // every piece of this stream is written: combine
+        const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
+        for (int e = tid; e < a.g * D; e += kThreads) {
           const int h = e / D, dd = e % D;
           float M = -INFINITY;
-          for (int c = first; c <= last; ++c)
-            M = fmaxf(M, __ldcg(a.part + (size_t)(c + i) * kMaxGroup * (D + 2) + kMaxGroup * D + h));
+#pragma unroll 4
+          for (int c = first; c <= last; ++c) M = fmaxf(M, __ldcg(&base[c].m[h]));
           float L = 0.f, O = 0.f;
+#pragma unroll 4
           for (int c = first; c <= last; ++c) {
-            const float* pc = a.part + (size_t)(c + i) * kMaxGroup * (D + 2);
-            const float sc = ex2(__ldcg(pc + kMaxGroup * D + h) - M);
-            L += __ldcg(pc + kMaxGroup * D + kMaxGroup + h) * sc;
-            O += __ldcg(pc + h * D + dd) * sc;
+            const float sc = ex2(__ldcg(&base[c].m[h]) - M);
+            L += __ldcg(&base[c].l[h]) * sc;
+            O += __ldcg(&base[c].O[h][dd]) * sc;
           }
           store_out(a, b, kvh * a.g + h, dd, D, O / L);
         }
         if (tid == 0) a.cnt[i] = 0;
       }
     }
-    named_barrier(1, NCW * 32);   // merge slots are reused by the next piece
+    __syncthreads();   // merge slots are reused by the next piece
     k = pe;
+    i = inext;
+    nn = nn_next;
   }
+
+  // Drain: copies issued but not consumed (only after an abort) must land before exit.
+  if (lane == 0)
+    for (int j = consumed; j < issued; ++j) mbar_wait_timed(smem_addr(&myfull[j % spw]), (j / spw) & 1, a.ctrl);
 }
 
 // ---------------------------------------------------------------------------
@@ -522,35 +613,25 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
 
 using KernelFn = void (*)(const AttnArgs, const __grid_constant__ CUtensorMap);
 
-struct Variant {
-  KernelFn fn;
-  int ncw, nstages, stage_bytes, d;
-};
+template <int D, int NCW, int NB, bool MMA, typename E>
+KernelFn kernel_ptr() { return attn_kernel<D, NCW, NB, MMA, E>; }
 
-constexpr int kNcw = 8;
-
-template <int D, int SPW, bool MMA, typename E>
-Variant make_variant() {
-  return Variant{attn_kernel<D, kNcw, SPW, MMA, E>, kNcw, kNcw * SPW, 2 * kPage * D * (int)sizeof(E), D};
+template <int NB, bool MMA, typename E>
+KernelFn pick_ncw(int d, int ncw) {
+  if (d == 64) return ncw == 4 ? kernel_ptr<64, 4, NB, MMA, E>() : kernel_ptr<64, 8, NB, MMA, E>();
+  return ncw == 4 ? kernel_ptr<128, 4, NB, MMA, E>() : kernel_ptr<128, 8, NB, MMA, E>();
 }
 
-bool pick_variant(int d, int dtype, int kernel, Variant* v) {
-  if (kernel == DMS_ATTN_MMA) {
-    if (dtype != DMS_BF16) return false;
-    *v = d == 64 ? make_variant<64, 2, true, uint16_t>() : make_variant<128, 2, true, uint16_t>();
-    return true;
-  }
-  if (dtype == DMS_BF16)
-    *v = d == 64 ? make_variant<64, 2, false, uint16_t>() : make_variant<128, 2, false, uint16_t>();
-  else
-    *v = d == 64 ? make_variant<64, 2, false, float>() : make_variant<128, 1, false, float>();
-  return true;
+KernelFn pick_kernel(int d, int dtype, int kernel, int ncw, int nb) {
+  if (kernel == DMS_ATTN_MMA)
+    return nb == 2 ? pick_ncw<2, true, uint16_t>(d, ncw) : pick_ncw<1, true, uint16_t>(d, ncw);
+  if (dtype == DMS_BF16) return pick_ncw<1, false, uint16_t>(d, ncw);
+  return pick_ncw<1, false, float>(d, ncw);
 }
 
-size_t smem_bytes(const Variant& v, int S) {
-  const size_t merge = (size_t)v.ncw * (kMaxGroup * (v.d + 2)) * sizeof(float);
-  return 1024 + (size_t)v.nstages * v.stage_bytes + 16 * (size_t)v.nstages + 64 + merge +
-         (size_t)(S + 1) * sizeof(int);
+int env_int(const char* name, int dflt) {
+  const char* v = getenv(name);
+  return (v && *v) ? atoi(v) : dflt;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -562,31 +643,55 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan) {
   int kernel = kernel_choice;
   if (kernel == DMS_ATTN_AUTO) kernel = (dtype == DMS_BF16) ? DMS_ATTN_MMA : DMS_ATTN_SIMT;
-  Variant v;
-  if (!pick_variant(dv.d, dtype, kernel, &v)) return cudaErrorInvalidValue;
+  if (kernel == DMS_ATTN_MMA && dtype != DMS_BF16) return cudaErrorInvalidValue;
+  // Tuning overrides: warps per CTA (4, 8), CTAs per SM (1, 2), stages per warp,
+  // pages per warp iteration (1, 2; tensor-core kernel only).
+  int ncw = env_int("DMS_ATTN_WARPS", 8);
+  if (ncw != 4) ncw = 8;
+  const int nb = (kernel == DMS_ATTN_MMA && env_int("DMS_ATTN_BATCH", 2) != 1) ? 2 : 1;
+  const int ctas = env_int("DMS_ATTN_CTAS", 1) == 2 ? 2 : 1;
+  const int stage_bytes = 2 * kPage * dv.d * dv.elem_bytes;
+  int dev = 0, per_sm_smem = 0, per_block_smem = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&per_sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&per_block_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  const int budget = std::min(per_block_smem, per_sm_smem / ctas - 1024) - 1024;   // minus alignment slack
+  const int fixed = smem_layout(ncw, 0, stage_bytes, dv.d, dv.S).total;
+  int spw = std::min(8, (budget - fixed) / (ncw * stage_bytes));
+  const int want = env_int("DMS_ATTN_STAGES", 0);
+  if (want > 0) spw = std::min(spw, want);
+  if (spw < nb) return cudaErrorInvalidConfiguration;
+
+  KernelFn fn = pick_kernel(dv.d, dtype, kernel, ncw, nb);
   plan->kernel = kernel;
-  plan->threads = (v.ncw + 1) * 32;
-  plan->smem = smem_bytes(v, dv.S);
-  cudaError_t e = cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan->smem);
+  plan->ncw = ncw;
+  plan->spw = spw;
+  plan->fn = reinterpret_cast<void*>(fn);
+  plan->threads = ncw * 32;
+  plan->smem = 1024 + (size_t)smem_layout(ncw, spw, stage_bytes, dv.d, dv.S).total;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan->smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, plan->threads, plan->smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, plan->threads, plan->smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  plan->grid = num_sms * per_sm;
+  plan->grid = num_sms * std::min(per_sm, ctas);
 
   memset(&plan->tmap, 0, sizeof(plan->tmap));
   if (kernel == DMS_ATTN_MMA) {
-    void* fn = nullptr;
+    void* enc = nullptr;
     cudaDriverEntryPointQueryResult q;
-    e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-    if (e != cudaSuccess || fn == nullptr || q != cudaDriverEntryPointSuccess) return cudaErrorNotSupported;
+    e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &enc, cudaEnableDefault, &q);
+    if (e != cudaSuccess || enc == nullptr || q != cudaDriverEntryPointSuccess) return cudaErrorNotSupported;
     // Pool viewed as [max_pages][32 rows][d] bf16; box = 64 columns x 32 rows of one page.
     const cuuint64_t dims[3] = {(cuuint64_t)dv.d, 32, (cuuint64_t)dv.max_pages};
     const cuuint64_t strides[2] = {(cuuint64_t)dv.d * 2, (cuuint64_t)dv.d * 2 * 32};
     const cuuint32_t box[3] = {64, 32, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = reinterpret_cast<EncodeTiledFn>(fn)(
+    CUresult r = reinterpret_cast<EncodeTiledFn>(enc)(
         &plan->tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dv.kv, dims, strides, box, estr,
         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -599,8 +704,6 @@ cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t s
                              const int32_t* seq_ids, const void* Q, int hq, float scale, void* out,
                              int out_f32) {
   if (n_seqs == 0) return cudaSuccess;
-  Variant v;
-  pick_variant(dv.d, dv.elem_bytes == 2 ? DMS_BF16 : DMS_F32, plan.kernel, &v);
   AttnArgs a;
   a.seq_ids = seq_ids;
   a.Q = (const uint8_t*)Q;
@@ -620,7 +723,9 @@ cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t s
   a.max_pages = dv.max_pages;
   a.out_f32 = out_f32;
   a.sl2e = scale * kLog2e;
-  v.fn<<<plan.grid, plan.threads, plan.smem, st>>>(a, plan.tmap);
+  a.spw = plan.spw;
+  a.S = dv.S;
+  reinterpret_cast<KernelFn>(plan.fn)<<<plan.grid, plan.threads, plan.smem, st>>>(a, plan.tmap);
   return cudaGetLastError();
 }
 

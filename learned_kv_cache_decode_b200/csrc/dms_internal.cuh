@@ -202,6 +202,7 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
 // ---------------------------------------------------------------------------
 // Host-side launchers (defined in dms_append.cu / dms_attention.cu).
 
+cudaError_t prepare_aux_kernels();
 cudaError_t launch_init_state(const Dev& dv, cudaStream_t st);
 cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
                                  const void* K, const void* V, const uint8_t* alpha, int* launches);
@@ -217,6 +218,9 @@ cudaError_t launch_gather(const Dev& dv, cudaStream_t st, int seq, int kvh, int 
 // Decode attention plan shared by host and launcher.
 struct AttnPlan {
   int kernel;        // DMS_ATTN_SIMT or DMS_ATTN_MMA
+  int ncw;           // warps per CTA, each with its own TMA page pipeline
+  int spw;           // shared-memory stages per warp
+  void* fn;          // kernel instantiation
   int grid;          // persistent CTAs
   int threads;
   size_t smem;       // dynamic shared memory bytes
