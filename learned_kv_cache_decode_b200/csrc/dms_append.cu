@@ -14,8 +14,8 @@ namespace dms {
 
 namespace {
 
-constexpr int kDecodeThreads = 128;
-constexpr int kDecodeStreamsPerBlock = 32;
+constexpr int kDecodeThreads = 1024;   // one block per decode append
+constexpr int kDecodePre = 4;          // 16-byte K/V vectors held in registers per thread
 
 __device__ __forceinline__ uint8_t* page_row(const Dev& dv, int page, int which, int row, int row_bytes) {
   return dv.kv + ((size_t)page * 2 * kPage + (size_t)which * kPage + row) * row_bytes;
@@ -29,135 +29,164 @@ __device__ __forceinline__ void warp_copy_row(uint8_t* dst, const uint8_t* src, 
 }
 
 // ---------------------------------------------------------------------------
-// Decode append: one token for each sequence of the call.
+// Decode append: one token for each stream of the call, in ONE block.
 //
-// Every block owns 32 streams (one lane of warp 0 each). A stream whose new
-// token reuses a retired slot or lands inside an already attached page is
-// finished by its own block. A stream whose token opens a new page is left
-// to the last block to arrive, which pops pages for all of them in stream
-// order, so page ids are deterministic without any inter-block waiting.
-__global__ void __launch_bounds__(kDecodeThreads)
+// A decode step appends a handful of rows, so the cost of this kernel is
+// its chain of dependent memory round trips, each a DRAM latency once the
+// attention has flushed L2 with pool reads. One block (no inter-block
+// hand-off, no grid-wide counter or fence) keeps the chain at four:
+//   1. status, free-stack depth, seq ids, alpha, and the new K/V rows
+//      (held in registers when they fit, else prefetched to L2);
+//   2. pos and n of every stream;
+//   3. the window-ring entry of the token that may leave (s - w);
+//   4. the page of the slot (page table), or a popped page for streams
+//      that open one (block scan in stream order, so pops are deterministic);
+// then the metadata stores and the row copies. Streams beyond the block
+// size go in rounds of kDecodeThreads, with the pop ranks carried over.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+__global__ void __launch_bounds__(kDecodeThreads, 1)
 append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
                      const uint8_t* __restrict__ K, const uint8_t* __restrict__ V,
                      const uint8_t* __restrict__ alpha) {
-  __shared__ int s_phys[kDecodeStreamsPerBlock];
+  extern __shared__ int s_phys[];   // [nst] physical slot that receives each stream's rows, -1 none
   __shared__ int s_warp[kDecodeThreads / 32];
-  __shared__ int s_last, s_ok;
+  constexpr int T = kDecodeThreads;
+  const int tid = threadIdx.x;
   const int nst = n_seqs * dv.hkv;
   const int row_bytes = dv.d * dv.elem_bytes;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int i0 = blockIdx.x * kDecodeStreamsPerBlock;
-  if (tid == 0) s_ok = (read_status(dv.ctrl) == 0);
-  __syncthreads();
-  const bool ok = s_ok;
+  const int chunks = row_bytes >> 4;              // 16-byte vectors per row
+  const int n_items = nst * 2 * chunks;           // (stream, K or V, vector)
 
-  if (tid < kDecodeStreamsPerBlock) {
-    const int i = i0 + tid;
-    int phys = -1;
-    if (ok && i < nst) {
-      int need = 0;
-      const int seq = seq_ids[i / dv.hkv];
-      if (seq < 0 || seq >= dv.max_seqs) {
-        latch(dv.ctrl, DMS_ERR_BAD_SEQ);
+  // ---- round trip 1
+  const int fc = *reinterpret_cast<const volatile int32_t*>(&dv.ctrl[kCtrlFree]);
+  auto item_src = [&](int t) -> const uint4* {
+    const int i = t / (2 * chunks), which = (t / chunks) & 1, c = t % chunks;
+    return reinterpret_cast<const uint4*>((which ? V : K) + (size_t)i * row_bytes) + c;
+  };
+  uint4 pre[kDecodePre];
+#pragma unroll
+  for (int p = 0; p < kDecodePre; ++p) {
+    const int t = tid + p * T;
+    if (t < n_items) pre[p] = __ldg(item_src(t));
+  }
+  for (int t = kDecodePre * T + tid * 8; t < n_items; t += 8 * T) prefetch_l2(item_src(t));   // 128-B lines
+  auto load_ids = [&](int i, int& seq, int& al) {
+    seq = -1;
+    al = 0;
+    if (i < nst) {
+      seq = __ldg(seq_ids + i / dv.hkv);
+      al = __ldg(alpha + i) != 0;
+    }
+  };
+  int seq, al;
+  load_ids(tid, seq, al);
+  if (__syncthreads_or(tid == 0 && read_status(dv.ctrl) != 0)) return;   // poisoned cache
+
+  // A call with more streams than threads learns its total page demand
+  // first, so that an exhausted pool fails every stream that needs a page.
+  int demand = -1;
+  if (nst > T) {
+    demand = 0;
+    for (int r0 = 0; r0 < nst; r0 += T) {
+      int sq, a_;
+      load_ids(r0 + tid, sq, a_);
+      bool need = false;
+      if (sq >= 0 && sq < dv.max_seqs) {
+        const int st = sq * dv.hkv + (r0 + tid) % dv.hkv;
+        const int s = dv.pos[st], nn = dv.n[st];
+        const int r = dv.ring[(size_t)st * dv.w + (s % dv.w)];
+        need = !((s >= dv.w) && (r & 1)) && (nn % kPage) == 0 && nn / kPage < dv.mps;
+      }
+      demand += __syncthreads_count(need);
+    }
+  }
+
+  int popped = 0;   // pages taken by earlier rounds
+  int failed = 0;   // pool exhausted
+  for (int r0 = 0; r0 < nst; r0 += T) {
+    const int i = r0 + tid;
+    const bool live = i < nst;
+    if (r0 > 0) load_ids(i, seq, al);
+    // ---- round trip 2
+    const bool good = live && seq >= 0 && seq < dv.max_seqs;
+    if (live && !good) latch(dv.ctrl, DMS_ERR_BAD_SEQ);
+    const int st = good ? seq * dv.hkv + i % dv.hkv : 0;
+    const int s = good ? dv.pos[st] : 0;
+    const int nn = good ? dv.n[st] : 0;
+    // ---- round trip 3
+    int32_t* rp = dv.ring + (size_t)st * dv.w + (s % dv.w);
+    const int r = good ? *rp : 0;
+    const bool retire = good && (s >= dv.w) && (r & 1);   // token s - w leaves now
+    const int slot = retire ? (r >> 1) : nn;
+    const int lp = slot / kPage;
+    bool go = good;
+    bool need = good && !retire && (slot % kPage) == 0;
+    if (need && lp >= dv.mps) {
+      latch(dv.ctrl, DMS_ERR_STREAM_FULL);
+      need = false;
+      go = false;
+    }
+    int total;
+    const int rank = block_exclusive_scan(need ? 1 : 0, s_warp, &total);
+    const bool fits = !failed && (demand >= 0 ? demand : total) <= fc;
+    if (!fits && total > 0) {
+      if (tid == 0) latch(dv.ctrl, DMS_ERR_POOL_EXHAUSTED);
+      failed = 1;
+    }
+    if (need && !fits) go = false;   // left unchanged: no stream of this round pops
+    // ---- round trip 4
+    int page = -1;
+    if (go) {
+      if (need) {
+        page = dv.free_list[fc - 1 - (popped + rank)];
       } else {
-        const int st = seq * dv.hkv + i % dv.hkv;
-        const int s = dv.pos[st];
-        int32_t* rp = dv.ring + (size_t)st * dv.w + (s % dv.w);
-        const int r = *rp;
-        const bool retire = (s >= dv.w) && (r & 1);   // token s - w leaves now
-        const int slot = retire ? (r >> 1) : dv.n[st];
-        if (!retire && (slot % kPage) == 0) {
-          need = 1;   // opens a page: finished by the last block
-        } else {
-          const int page = slot / kPage < dv.mps ? dv.page_table[(size_t)st * dv.mps + slot / kPage] : -1;
-          if (page < 0 || page >= dv.max_pages) {
-            latch(dv.ctrl, DMS_ERR_INVALID);
-          } else {
-            if (!retire) dv.n[st] = slot + 1;
-            phys = page * kPage + slot % kPage;
-            *rp = (slot << 1) | (alpha[i] != 0);
-            dv.pos[st] = s + 1;
-            dv.slot_pos[phys] = s;
-          }
+        page = dv.page_table[(size_t)st * dv.mps + lp];
+        if (page < 0 || page >= dv.max_pages) {
+          latch(dv.ctrl, DMS_ERR_INVALID);
+          go = false;
         }
       }
-      dv.scratch[i] = need;
     }
-    s_phys[tid] = phys;
-  }
-  __syncthreads();
-
-  // K and V rows of the streams finished here (warp per stream).
-  for (int l = warp; l < kDecodeStreamsPerBlock; l += kDecodeThreads / 32) {
-    const int phys = s_phys[l];
-    if (phys < 0) continue;
-    const size_t src = (size_t)(i0 + l) * row_bytes;
-    warp_copy_row(page_row(dv, phys / kPage, 0, phys % kPage, row_bytes), K + src, row_bytes, lane);
-    warp_copy_row(page_row(dv, phys / kPage, 1, phys % kPage, row_bytes), V + src, row_bytes, lane);
-  }
-
-  // Last block to arrive pops pages for the deferred streams.
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&dv.ctrl[kCtrlArrive], 1) == (int)gridDim.x - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  const bool still_ok = ok && read_status(dv.ctrl) == 0;
-  const int per = (nst + kDecodeThreads - 1) / kDecodeThreads;
-  const int b = min(tid * per, nst), e = min(b + per, nst);
-  int cnt = 0;
-  if (still_ok)
-    for (int i = b; i < e; ++i) cnt += __ldcg(&dv.scratch[i]);
-  int total;
-  int rank = block_exclusive_scan(cnt, s_warp, &total);
-  const int fc = *reinterpret_cast<volatile int32_t*>(&dv.ctrl[kCtrlFree]);
-  const bool fits = still_ok && total <= fc;
-  if (still_ok && !fits && tid == 0) latch(dv.ctrl, DMS_ERR_POOL_EXHAUSTED);
-  if (fits && total > 0) {
-    for (int i = b; i < e; ++i) {
-      if (__ldcg(&dv.scratch[i]) == 0) continue;
-      const int page = dv.free_list[fc - 1 - rank];
-      ++rank;
-      const int st = seq_ids[i / dv.hkv] * dv.hkv + i % dv.hkv;
-      const int s = dv.pos[st];
-      const int slot = dv.n[st];
-      const int lp = slot / kPage;
-      if (lp >= dv.mps) {
-        latch(dv.ctrl, DMS_ERR_STREAM_FULL);
-        dv.scratch[i] = 0;
-        continue;
+    int phys = -1;
+    if (go) {
+      if (need) {
+        dv.page_table[(size_t)st * dv.mps + lp] = page;
+        dv.n_pages[st] = lp + 1;
       }
-      dv.page_table[(size_t)st * dv.mps + lp] = page;
-      dv.n_pages[st] = lp + 1;
-      dv.n[st] = slot + 1;
-      dv.ring[(size_t)st * dv.w + (s % dv.w)] = (slot << 1) | (alpha[i] != 0);
+      if (!retire) dv.n[st] = slot + 1;
+      phys = page * kPage + slot % kPage;
+      *rp = (slot << 1) | al;
       dv.pos[st] = s + 1;
-      dv.slot_pos[page * kPage] = s;
-      dv.scratch[i] = -(page + 1);   // row copy below
+      dv.slot_pos[phys] = s;
     }
+    if (live) s_phys[i] = phys;
+    if (fits) popped += total;
   }
+  if (tid == 0 && popped > 0) dv.ctrl[kCtrlFree] = fc - popped;
   __syncthreads();
-  if (fits && total > 0) {
-    // Copy rows of the deferred streams, warp per stream.
-    for (int base = warp * 32; base < nst; base += kDecodeThreads) {
-      const int i = base + lane;
-      const int v = (i < nst) ? __ldcg(&dv.scratch[i]) : 0;
-      unsigned mask = __ballot_sync(0xffffffffu, v < 0);
-      while (mask) {
-        const int l = __ffs(mask) - 1;
-        mask &= mask - 1;
-        const int page = -__shfl_sync(0xffffffffu, v, l) - 1;
-        const size_t src = (size_t)(base + l) * row_bytes;
-        warp_copy_row(page_row(dv, page, 0, 0, row_bytes), K + src, row_bytes, lane);
-        warp_copy_row(page_row(dv, page, 1, 0, row_bytes), V + src, row_bytes, lane);
-      }
+
+  // ---- K and V rows into their slots: 16-byte vectors, consecutive threads
+  // on consecutive vectors of a row.
+  auto item_dst = [&](int t, int phys) -> uint4* {
+    const int which = (t / chunks) & 1, c = t % chunks;
+    const int page = phys / kPage, row = phys % kPage;
+    return reinterpret_cast<uint4*>(dv.kv + ((size_t)page * 2 * kPage + (size_t)which * kPage + row) * row_bytes) + c;
+  };
+#pragma unroll
+  for (int p = 0; p < kDecodePre; ++p) {
+    const int t = tid + p * T;
+    if (t < n_items) {
+      const int phys = s_phys[t / (2 * chunks)];
+      if (phys >= 0) *item_dst(t, phys) = pre[p];
     }
   }
-  if (tid == 0) {
-    if (fits) dv.ctrl[kCtrlFree] = fc - total;
-    dv.ctrl[kCtrlArrive] = 0;
+#pragma unroll 4
+  for (int t = kDecodePre * T + tid; t < n_items; t += T) {
+    const int phys = s_phys[t / (2 * chunks)];
+    if (phys >= 0) *item_dst(t, phys) = __ldg(item_src(t));
   }
 }
 
@@ -444,9 +473,8 @@ cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, con
                                  const void* K, const void* V, const uint8_t* alpha, int* launches) {
   const int nst = n_seqs * dv.hkv;
   if (nst == 0) return cudaSuccess;
-  const int blocks = (nst + kDecodeStreamsPerBlock - 1) / kDecodeStreamsPerBlock;
-  append_decode_kernel<<<blocks, kDecodeThreads, 0, st>>>(dv, n_seqs, seq_ids, (const uint8_t*)K,
-                                                         (const uint8_t*)V, alpha);
+  append_decode_kernel<<<1, kDecodeThreads, (size_t)nst * sizeof(int), st>>>(
+      dv, n_seqs, seq_ids, (const uint8_t*)K, (const uint8_t*)V, alpha);
   *launches += 1;
   return cudaGetLastError();
 }

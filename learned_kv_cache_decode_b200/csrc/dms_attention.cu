@@ -346,6 +346,20 @@ __device__ __forceinline__ void store_out(const AttnArgs& a, int b, int h, int d
   }
 }
 
+// Store 4 consecutive output elements (v * inv) of query head h at dims [dd, dd + 4).
+__device__ __forceinline__ void store_out4(const AttnArgs& a, int b, int h, int dd, int D, float4 v, float inv) {
+  const size_t idx = ((size_t)b * a.hq + h) * D + dd;
+  if (a.out_f32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + idx) =
+        make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+  } else {
+    uint2 r;
+    r.x = pack_bf16x2(v.x * inv, v.y * inv);
+    r.y = pack_bf16x2(v.z * inv, v.w * inv);
+    *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + idx) = r;
+  }
+}
+
 // Shared-memory layout of one CTA (byte offsets from a 1024-aligned base).
 struct SmemLayout {
   int stages, bars, misc, merge, prefix, sid, total;
@@ -544,57 +558,92 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     const int nn_next = pe < K1 ? __ldg(a.n + sid[inext]) : 0;
     __syncthreads();
 
+    // Merge: thread t owns query head h = t / (D/4) and dims [4 d4, 4 d4 + 4);
+    // the CTA's result for its items stays in registers for the combine.
+    constexpr int kItems = kMaxGroup * D / 4;
+    constexpr int kIters = (kItems + kThreads - 1) / kThreads;
+    const int items = a.g * (D / 4);
+    float4 myO[kIters];
+    float myM[kIters], myL[kIters];
     Partial<D>* part = reinterpret_cast<Partial<D>*>(a.part) + (blockIdx.x + i);
-    for (int e = tid; e < a.g * D; e += kThreads) {
-      const int h = e / D, dd = e % D;
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      const int t = tid + it * kThreads;
+      if (t >= items) break;
+      const int h = t / (D / 4), d4 = t % (D / 4);
       float M = -INFINITY;
 #pragma unroll
       for (int w = 0; w < NCW; ++w) M = fmaxf(M, slots[w].m[h]);
-      float L = 0.f, O = 0.f;
+      float L = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int w = 0; w < NCW; ++w) {
-        const float mw = slots[w].m[h];
-        if (mw == -INFINITY) continue;
-        const float sc = ex2(mw - M);
-        L += slots[w].l[h] * sc;
-        O += slots[w].O[h][dd] * sc;
+        const float sc = ex2(slots[w].m[h] - M);   // 0 for a warp that saw nothing (m = -inf)
+        const float4 o = *reinterpret_cast<const float4*>(&slots[w].O[h][4 * d4]);
+        L = fmaf(slots[w].l[h], sc, L);
+        O.x = fmaf(o.x, sc, O.x);
+        O.y = fmaf(o.y, sc, O.y);
+        O.z = fmaf(o.z, sc, O.z);
+        O.w = fmaf(o.w, sc, O.w);
       }
       if (whole) {
-        store_out(a, b, kvh * a.g + h, dd, D, O / L);
+        store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, 1.f / L);
       } else {
-        part->O[h][dd] = O;
-        if (dd == 0) {
-          part->m[h] = M;
-          part->l[h] = L;
+        __stcg(reinterpret_cast<float4*>(&part->O[h][4 * d4]), O);
+        if (d4 == 0) {
+          __stcg(&part->m[h], M);
+          __stcg(&part->l[h], L);
         }
+        myO[it] = O;
+        myM[it] = M;
+        myL[it] = L;
       }
     }
     if (!whole) {
-      __syncthreads();   // the partial is complete in this CTA ...
-      const int first = range_of(pstart, P, Geff), last = range_of(pend - 1, P, Geff);
-      if (tid == 0) {
-        __threadfence();   // ... and visible device-wide before the count moves
-        misc[2] = (atomicAdd(&a.cnt[i], 1) == last - first);
-        if (misc[2]) __threadfence();
-      }
+      // Publish the partial: the CTA's stores, ordered by the barrier, are
+      // released by thread 0's device-scope add; the adder that completes the
+      // count acquires every other piece and combines.
       __syncthreads();
-      if (misc[2]) {   // every piece of this stream is written: combine
+      const int first = range_of(pstart, P, Geff), last = range_of(pend - 1, P, Geff);
+      if (tid == 0) misc[2] = (atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first);
+      __syncthreads();
+      if (misc[2]) {
         const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
-        for (int e = tid; e < a.g * D; e += kThreads) {
-          const int h = e / D, dd = e % D;
-          float M = -INFINITY;
-#pragma unroll 4
-          for (int c = first; c <= last; ++c) M = fmaxf(M, __ldcg(&base[c].m[h]));
-          float L = 0.f, O = 0.f;
-#pragma unroll 4
-          for (int c = first; c <= last; ++c) {
-            const float sc = ex2(__ldcg(&base[c].m[h]) - M);
-            L += __ldcg(&base[c].l[h]) * sc;
-            O += __ldcg(&base[c].O[h][dd]) * sc;
+        const int me = blockIdx.x;
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+          const int t = tid + it * kThreads;
+          if (t >= items) break;
+          const int h = t / (D / 4), d4 = t % (D / 4);
+          float M = myM[it], L = myL[it];
+          float4 O = myO[it];
+          for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
+            float mc[4], lc[4];
+            float4 oc[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int c = c0 + u;
+              const bool use = c <= last && c != me;
+              mc[u] = use ? __ldcg(&base[c].m[h]) : -INFINITY;
+              lc[u] = use ? __ldcg(&base[c].l[h]) : 0.f;
+              oc[u] = use ? __ldcg(reinterpret_cast<const float4*>(&base[c].O[h][4 * d4]))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float Mn = fmaxf(M, mc[u]);
+              const float sa = ex2(M - Mn), sb = ex2(mc[u] - Mn);
+              L = L * sa + lc[u] * sb;
+              O.x = O.x * sa + oc[u].x * sb;
+              O.y = O.y * sa + oc[u].y * sb;
+              O.z = O.z * sa + oc[u].z * sb;
+              O.w = O.w * sa + oc[u].w * sb;
+              M = Mn;
+            }
           }
-          store_out(a, b, kvh * a.g + h, dd, D, O / L);
+          store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, 1.f / L);
         }
-        if (tid == 0) a.cnt[i] = 0;
+        if (tid == 0) a.cnt[i] = 0;   // ready for the next launch (stream order)
       }
     }
     __syncthreads();   // merge slots are reused by the next piece
