@@ -173,6 +173,67 @@ dms_status dms_snapshot(dms_cache* cache, cudaStream_t stream, int32_t* page_tab
 dms_status dms_gather_kv(dms_cache* cache, cudaStream_t stream, int32_t seq_id,
                          int32_t kv_head, int32_t rows_cap, void* K_out, void* V_out);
 
+/* ---- Decode attention that allocates nothing ---------------------------
+ * The paper has no counterpart to this call. It is for callers that must
+ * not allocate device memory while they decode: a framework whose caching
+ * allocator already holds the device memory (a cudaMalloc of its own could
+ * fail or synchronise the device), or a runtime that owns every buffer and
+ * lends the library its K/V pages. dms_decode_attention cannot serve them,
+ * because its scratch comes with a dms_cache, and dms_cache_create
+ * allocates.
+ *
+ * Same arithmetic and kernels as dms_decode_attention, over K/V pages the
+ * caller owns and lays out as a dms_cache does (see "Storage" above). The
+ * split-K scratch (partials, arrival counters, status word) is a static
+ * device array of about 4.1 MiB inside the library. The CUDA runtime
+ * places it on each device that loads the library and keeps it until the
+ * process exits. The call itself makes no cudaMalloc, cudaFree or other
+ * allocating call.
+ *
+ * The first call on a device (with that device current) looks up the
+ * array's device address and sets the kernel's attributes. Make that first
+ * call before any stream capture. Later calls reuse the set-up.
+ *
+ * Every call on a device shares the one array: calls whose kernels may
+ * overlap on the GPU (different streams, no ordering between them) race on
+ * it and give wrong results. Each call clears the counters and status word
+ * it uses on `stream` (cudaMemsetAsync) before its kernel.
+ *
+ * Limits: n_seqs * num_kv_heads <= DMS_NOALLOC_MAX_STREAMS, and the grid
+ * (one CTA per SM) plus the streams <= DMS_NOALLOC_MAX_PIECES. Beyond them
+ * the call returns DMS_ERR_INVALID and launches nothing.
+ *
+ *   kv           host pointer to the description of the caller's cache:
+ *     kv_pool      device [max_pages][2][16][head_dim] of dtype, 16-B aligned:
+ *                  per page 16 K rows then 16 V rows
+ *     page_table   device int32 [max_seqs * num_kv_heads][max_pages_per_stream]
+ *     retained     device int32 [max_seqs * num_kv_heads]: n of each stream,
+ *                  in [0, 16 * max_pages_per_stream]; its tokens sit in
+ *                  logical slots [0, n). Larger or negative counts are not
+ *                  checked and make the kernel read past the page table.
+ *   seq_ids, Q, num_q_heads, scale, out, out_dtype: as dms_decode_attention.
+ * Device-side checks (a seq id outside [0, max_seqs), a page id outside
+ * [0, max_pages)) skip the bad access, but no later call reports them: the
+ * outputs of those streams are then unspecified. Async. */
+#define DMS_NOALLOC_MAX_STREAMS 512
+#define DMS_NOALLOC_MAX_PIECES 1024
+
+typedef struct {
+    const void* kv_pool;
+    const int32_t* page_table;
+    const int32_t* retained;
+    int32_t max_seqs;
+    int32_t num_kv_heads;
+    int32_t head_dim;              /* 64 or 128 */
+    int32_t max_pages;
+    int32_t max_pages_per_stream;
+    dms_dtype dtype;               /* storage type of K, V and Q */
+} dms_paged_kv;
+
+dms_status dms_decode_attention_noalloc(cudaStream_t stream, const dms_paged_kv* kv, int32_t n_seqs,
+                                        const int32_t* seq_ids, const void* Q, int32_t num_q_heads,
+                                        float scale, void* out, dms_dtype out_dtype);
+
 /* Sync the stream and return the latched device status (DMS_OK if none). */
 dms_status dms_get_status(dms_cache* cache, cudaStream_t stream);
 

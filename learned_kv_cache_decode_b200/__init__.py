@@ -21,7 +21,7 @@ import torch
 from . import _native
 from ._native import DmsError
 
-__all__ = ["DmsCache", "DmsError"]
+__all__ = ["DmsCache", "DmsError", "decode_attention_noalloc"]
 
 _DTYPES = {torch.bfloat16: _native.DMS_BF16, torch.float32: _native.DMS_F32}
 _KERNELS = {"auto": _native.DMS_ATTN_AUTO, "simt": _native.DMS_ATTN_SIMT, "mma": _native.DMS_ATTN_MMA}
@@ -151,3 +151,30 @@ class DmsCache:
 
     def launches(self) -> int:
         return int(self.lib.dms_launch_count(self._h))
+
+
+def decode_attention_noalloc(kv_pool: torch.Tensor, page_table: torch.Tensor, retained: torch.Tensor,
+                             num_kv_heads: int, seq_ids: torch.Tensor, Q: torch.Tensor,
+                             scale: float | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode attention over caller-owned paged K/V; the library allocates nothing
+    (wraps ``dms_decode_attention_noalloc``).
+
+    kv_pool [max_pages, 2, 16, d] (K rows then V rows per page), page_table int32
+    [max_seqs * num_kv_heads, max_pages_per_stream], retained int32 [max_seqs *
+    num_kv_heads], seq_ids int32 [B], Q [B, Hq, d] -> out [B, Hq, d]. ``out`` must be
+    passed by a caller that may not allocate.
+    """
+    lib = _native.load()
+    b, hq, d = Q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((b, hq, d), dtype=Q.dtype, device=Q.device)
+    streams, mps = page_table.shape
+    kv = _native.DmsPagedKv(kv_pool.data_ptr(), page_table.data_ptr(), retained.data_ptr(),
+                            streams // num_kv_heads, num_kv_heads, d, kv_pool.shape[0], mps,
+                            _DTYPES[kv_pool.dtype])
+    _native.check(lib.dms_decode_attention_noalloc(_stream(), ctypes.byref(kv), int(seq_ids.numel()),
+                                                   _ptr(seq_ids), _ptr(Q), hq, float(scale), _ptr(out),
+                                                   _DTYPES[out.dtype]), "dms_decode_attention_noalloc")
+    return out

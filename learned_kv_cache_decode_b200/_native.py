@@ -29,7 +29,10 @@ DMS_ATTN_MMA = 2
 
 EXPORTS = ("dms_cache_create", "dms_cache_destroy", "dms_cache_reset", "dms_seq_reset", "dms_append",
            "dms_decode_attention", "dms_stats", "dms_snapshot", "dms_gather_kv", "dms_get_status",
-           "dms_status_string", "dms_launch_count")
+           "dms_status_string", "dms_launch_count", "dms_decode_attention_noalloc")
+
+DMS_NOALLOC_MAX_STREAMS = 512
+DMS_NOALLOC_MAX_PIECES = 1024
 
 
 class DmsConfig(ctypes.Structure):
@@ -43,6 +46,21 @@ class DmsConfig(ctypes.Structure):
         ("max_pages_per_stream", ctypes.c_int32),
         ("dtype", ctypes.c_int),
         ("attn_kernel", ctypes.c_int),
+    ]
+
+
+class DmsPagedKv(ctypes.Structure):
+    """Caller-owned paged K/V for dms_decode_attention_noalloc."""
+    _fields_ = [
+        ("kv_pool", ctypes.c_void_p),
+        ("page_table", ctypes.c_void_p),
+        ("retained", ctypes.c_void_p),
+        ("max_seqs", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("max_pages", ctypes.c_int32),
+        ("max_pages_per_stream", ctypes.c_int32),
+        ("dtype", ctypes.c_int),
     ]
 
 
@@ -91,6 +109,9 @@ def load() -> ctypes.CDLL:
     L.dms_status_string.restype = ctypes.c_char_p
     L.dms_launch_count.argtypes = [p]
     L.dms_launch_count.restype = i64
+    L.dms_decode_attention_noalloc.argtypes = [p, ctypes.POINTER(DmsPagedKv), i32, p, p, i32, ctypes.c_float, p,
+                                               ctypes.c_int]
+    L.dms_decode_attention_noalloc.restype = st
     _lib = L
     return L
 

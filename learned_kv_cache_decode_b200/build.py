@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdms.so")
-SOURCES = ["dms_api.cu", "dms_append.cu", "dms_attention.cu"]
+SOURCES = ["dms_api.cu", "dms_append.cu", "dms_attention.cu", "dms_noalloc.cu"]
 HEADERS = [os.path.join(CSRC, "dms_internal.cuh"), os.path.join(INCLUDE, "dms.h")]
 
 NVCC_FLAGS = [
