@@ -60,6 +60,11 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
   const int chunks = row_bytes >> 4;              // 16-byte vectors per row
   const int n_items = nst * 2 * chunks;           // (stream, K or V, vector)
 
+  // Launched early behind the previous kernel of the stream (programmatic
+  // dependent launch): nothing is read before this wait.
+  grid_dependency_wait();
+  grid_dependents_launch();
+
   // ---- round trip 1
   const int fc = *reinterpret_cast<const volatile int32_t*>(&dv.ctrl[kCtrlFree]);
   auto item_src = [&](int t) -> const uint4* {
@@ -473,10 +478,9 @@ cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, con
                                  const void* K, const void* V, const uint8_t* alpha, int* launches) {
   const int nst = n_seqs * dv.hkv;
   if (nst == 0) return cudaSuccess;
-  append_decode_kernel<<<1, kDecodeThreads, (size_t)nst * sizeof(int), st>>>(
-      dv, n_seqs, seq_ids, (const uint8_t*)K, (const uint8_t*)V, alpha);
   *launches += 1;
-  return cudaGetLastError();
+  return launch_dependent(append_decode_kernel, dim3(1), dim3(kDecodeThreads), (size_t)nst * sizeof(int), st, dv,
+                          n_seqs, seq_ids, (const uint8_t*)K, (const uint8_t*)V, alpha);
 }
 
 cudaError_t launch_append_bulk(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,

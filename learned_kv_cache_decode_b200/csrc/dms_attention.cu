@@ -97,16 +97,32 @@ struct MmaState {
   float m[2], l[2];
 };
 
+// Query of one stream, as this lane's Q^T B-fragments.
 template <int D>
-__device__ __forceinline__ void mma_load_q(MmaState<D>& S, const AttnArgs& a, int b, int kvh, int lane) {
+struct MmaQuery {
+  uint32_t qb[D / 16][2];
+};
+
+template <int D>
+__device__ __forceinline__ void mma_fetch_q(MmaQuery<D>& Q, const AttnArgs& a, int b, int kvh, int lane) {
   const int n = lane >> 2;                 // head column of this lane's B fragment
   const bool live = n < a.g;
   const uint32_t* q = reinterpret_cast<const uint32_t*>(
       a.Q + ((size_t)b * a.hq + (size_t)kvh * a.g + (live ? n : 0)) * D * 2);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    S.qb[kk][0] = live ? __ldg(q + kk * 8 + (lane & 3)) : 0u;
-    S.qb[kk][1] = live ? __ldg(q + kk * 8 + 4 + (lane & 3)) : 0u;
+    Q.qb[kk][0] = live ? __ldg(q + kk * 8 + (lane & 3)) : 0u;
+    Q.qb[kk][1] = live ? __ldg(q + kk * 8 + 4 + (lane & 3)) : 0u;
+  }
+}
+
+// Start a piece: take its query, clear the softmax state.
+template <int D>
+__device__ __forceinline__ void mma_start(MmaState<D>& S, const MmaQuery<D>& Q) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    S.qb[kk][0] = Q.qb[kk][0];
+    S.qb[kk][1] = Q.qb[kk][1];
   }
 #pragma unroll
   for (int mt = 0; mt < D / 16; ++mt)
@@ -280,16 +296,32 @@ __device__ __forceinline__ void simt_load_row(const E* row, int lane, float (&x)
   for (int e = 0; e < D / 32; ++e) x[e] = to_f32<E>(row[lane * (D / 32) + e]);
 }
 
+// Query of one stream, this lane's head_dim slice of every head, pre-scaled
+// by scale * log2(e).
+template <int D>
+struct SimtQuery {
+  float q[kMaxGroup][D / 32];
+};
+
 template <int D, typename E>
-__device__ __forceinline__ void simt_load_q(SimtState<D>& S, const AttnArgs& a, int b, int kvh, int lane) {
+__device__ __forceinline__ void simt_fetch_q(SimtQuery<D>& Q, const AttnArgs& a, int b, int kvh, int lane) {
   const E* q = reinterpret_cast<const E*>(a.Q) + ((size_t)b * a.hq + (size_t)kvh * a.g) * D;
 #pragma unroll
   for (int h = 0; h < kMaxGroup; ++h) {
     float x[D / 32];
     if (h < a.g) simt_load_row<D, E>(q + (size_t)h * D, lane, x);
 #pragma unroll
+    for (int e = 0; e < D / 32; ++e) Q.q[h][e] = h < a.g ? x[e] * a.sl2e : 0.f;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void simt_start(SimtState<D>& S, const SimtQuery<D>& Q) {
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h) {
+#pragma unroll
     for (int e = 0; e < D / 32; ++e) {
-      S.q[h][e] = h < a.g ? x[e] * a.sl2e : 0.f;
+      S.q[h][e] = Q.q[h][e];
       S.acc[h][e] = 0.f;
     }
     S.m[h] = -INFINITY;
@@ -360,6 +392,19 @@ __device__ __forceinline__ void store_out4(const AttnArgs& a, int b, int h, int 
   }
 }
 
+// Online merge of partial (m2, l2, o2) into (m, l, o); scores in base 2.
+// At least one of m, m2 must be finite.
+__device__ __forceinline__ void merge_into(float& m, float& l, float4& o, float m2, float l2, float4 o2) {
+  const float mn = fmaxf(m, m2);
+  const float sa = ex2(m - mn), sb = ex2(m2 - mn);   // 0 for a side that saw nothing (m = -inf)
+  l = l * sa + l2 * sb;
+  o.x = o.x * sa + o2.x * sb;
+  o.y = o.y * sa + o2.y * sb;
+  o.z = o.z * sa + o2.z * sb;
+  o.w = o.w * sa + o2.w * sb;
+  m = mn;
+}
+
 // Shared-memory layout of one CTA (byte offsets from a 1024-aligned base).
 struct SmemLayout {
   int stages, bars, misc, merge, prefix, sid, total;
@@ -397,7 +442,9 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   const int spw = a.spw;
   const SmemLayout lay = smem_layout(NCW, spw, kStage, D, a.S);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
-  int* misc = reinterpret_cast<int*>(smem + lay.misc);   // [0] abort, [1] ok, [2] last, [3..] scan scratch
+  // misc: [0] abort, [1] ok, [2] last flag, [3 .. 3+NCW] scan scratch,
+  // [14] stream whose combine a split first piece left to the end of the range (-1: none)
+  int* misc = reinterpret_cast<int*>(smem + lay.misc);
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(smem + lay.merge);
   int* prefix = reinterpret_cast<int*>(smem + lay.prefix);
   int* sid = reinterpret_cast<int*>(smem + lay.sid);
@@ -408,15 +455,19 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
 
   if (tid == 0) {
     misc[0] = 0;
-    misc[1] = (read_status(a.ctrl) == 0);
+    misc[14] = -1;
     for (int s = 0; s < NCW * spw; ++s) mbar_init(smem_addr(&full[s]), 1);
     fence_mbar_init();
   }
-  __syncthreads();
-  if (!misc[1]) return;   // poisoned cache: do nothing
+  // Launched early behind the previous kernel of the stream (programmatic
+  // dependent launch): everything above overlaps it; nothing it writes is
+  // read before this point.
+  grid_dependency_wait();
 
-  // ---- plan: retained pages per stream of the call (prefix) and stream ids, in smem
+  // ---- plan: retained pages per stream of the call (prefix) and stream ids,
+  // in smem. The status word is read in the same round trip as the seq ids.
   {
+    const int status = tid == 0 ? read_status(a.ctrl) : 0;
     const int per = (nst + kThreads - 1) / kThreads;
     const int b0 = min(tid * per, nst), e0 = min(b0 + per, nst);
     int local = 0;
@@ -439,9 +490,14 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       run += prefix[i + 1];
       prefix[i + 1] = run;
     }
-    if (tid == 0) prefix[0] = 0;
+    if (tid == 0) {
+      prefix[0] = 0;
+      misc[1] = (status == 0);
+    }
   }
   __syncthreads();
+  grid_dependents_launch();   // the next kernel may queue up behind this one
+  if (!misc[1]) return;   // poisoned cache: do nothing (uniform over the CTA)
   const long long P = prefix[nst];
   const int G = gridDim.x;
 
@@ -499,13 +555,23 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   for (int j = 0; j < spw && j < njobs; ++j) issue(j);
 
   using State = typename std::conditional<MMA, MmaState<D>, SimtState<D>>::type;
+  using Query = typename std::conditional<MMA, MmaQuery<D>, SimtQuery<D>>::type;
   State S;
+  Query qcur;
+  auto load_query = [&](int stream) {   // the piece's query; clears the softmax state
+    if constexpr (MMA) {
+      mma_fetch_q<D>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
+      mma_start<D>(S, qcur);
+    } else {
+      simt_fetch_q<D, E>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
+      simt_start<D>(S, qcur);
+    }
+  };
   const MmaOffsets<D> off(lane);
   int consumed = 0;
   int k = K0;
   int i = stream_of(prefix, nst, k);
-  if constexpr (MMA) mma_load_q<D>(S, a, i / a.hkv, i % a.hkv, lane);
-  else simt_load_q<D, E>(S, a, i / a.hkv, i % a.hkv, lane);
+  load_query(i);
   int nn = __ldg(a.n + sid[i]);
   while (k < K1) {
     const int pstart = prefix[i], pend = prefix[i + 1];
@@ -551,10 +617,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     else simt_to_slot<D>(S, &slots[warp], lane);
     // start loading the next piece's query while the CTA merges
     const int inext = pe < K1 ? stream_of(prefix, nst, pe) : i;
-    if (pe < K1) {
-      if constexpr (MMA) mma_load_q<D>(S, a, inext / a.hkv, inext % a.hkv, lane);
-      else simt_load_q<D, E>(S, a, inext / a.hkv, inext % a.hkv, lane);
-    }
+    if (pe < K1) load_query(inext);
     const int nn_next = pe < K1 ? __ldg(a.n + sid[inext]) : 0;
     __syncthreads();
 
@@ -599,57 +662,86 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
         myL[it] = L;
       }
     }
+    __syncthreads();   // the slots are read and the partial (if any) is complete
     if (!whole) {
       // Publish the partial: the CTA's stores, ordered by the barrier, are
       // released by thread 0's device-scope add; the adder that completes the
       // count acquires every other piece and combines.
-      __syncthreads();
       const int first = range_of(pstart, P, Geff), last = range_of(pend - 1, P, Geff);
-      if (tid == 0) misc[2] = (atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first);
-      __syncthreads();
-      if (misc[2]) {
-        const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
-        const int me = blockIdx.x;
+      if (pe < K1) {
+        // A split piece inside the range is its first piece. Thread 0
+        // publishes it while the CTA goes on; a combine it finds due is done
+        // by the whole CTA at the end of the range.
+        if (tid == 0 && atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first) misc[14] = i;
+      } else {
+        if (tid == 0) misc[2] = (atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first);
+        __syncthreads();
+        if (misc[2]) {
+          const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
+          const int me = blockIdx.x;
 #pragma unroll
-        for (int it = 0; it < kIters; ++it) {
-          const int t = tid + it * kThreads;
-          if (t >= items) break;
-          const int h = t / (D / 4), d4 = t % (D / 4);
-          float M = myM[it], L = myL[it];
-          float4 O = myO[it];
-          for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
-            float mc[4], lc[4];
-            float4 oc[4];
+          for (int it = 0; it < kIters; ++it) {
+            const int t = tid + it * kThreads;
+            if (t >= items) break;
+            const int h = t / (D / 4), d4 = t % (D / 4);
+            float M = myM[it], L = myL[it];
+            float4 O = myO[it];
+            for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
+              float mc[4], lc[4];
+              float4 oc[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int c = c0 + u;
-              const bool use = c <= last && c != me;
-              mc[u] = use ? __ldcg(&base[c].m[h]) : -INFINITY;
-              lc[u] = use ? __ldcg(&base[c].l[h]) : 0.f;
-              oc[u] = use ? __ldcg(reinterpret_cast<const float4*>(&base[c].O[h][4 * d4]))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+              for (int u = 0; u < 4; ++u) {
+                const int c = c0 + u;
+                const bool use = c <= last && c != me;
+                mc[u] = use ? __ldcg(&base[c].m[h]) : -INFINITY;
+                lc[u] = use ? __ldcg(&base[c].l[h]) : 0.f;
+                oc[u] = use ? __ldcg(reinterpret_cast<const float4*>(&base[c].O[h][4 * d4]))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u) merge_into(M, L, O, mc[u], lc[u], oc[u]);
             }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float Mn = fmaxf(M, mc[u]);
-              const float sa = ex2(M - Mn), sb = ex2(mc[u] - Mn);
-              L = L * sa + lc[u] * sb;
-              O.x = O.x * sa + oc[u].x * sb;
-              O.y = O.y * sa + oc[u].y * sb;
-              O.z = O.z * sa + oc[u].z * sb;
-              O.w = O.w * sa + oc[u].w * sb;
-              M = Mn;
-            }
+            store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, 1.f / L);
           }
-          store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, 1.f / L);
+          if (tid == 0) a.cnt[i] = 0;   // ready for the next launch (stream order)
         }
-        if (tid == 0) a.cnt[i] = 0;   // ready for the next launch (stream order)
       }
     }
-    __syncthreads();   // merge slots are reused by the next piece
     k = pe;
     i = inext;
     nn = nn_next;
+  }
+
+  // ---- a split first piece that completed its stream: combine all its pieces
+  __syncthreads();
+  if (misc[14] >= 0) {
+    const int i = misc[14];
+    const int first = range_of(prefix[i], P, Geff), last = range_of(prefix[i + 1] - 1, P, Geff);
+    const int b = i / a.hkv, kvh = i % a.hkv;
+    const int items = a.g * (D / 4);
+    const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
+    for (int t = tid; t < items; t += kThreads) {
+      const int h = t / (D / 4), d4 = t % (D / 4);
+      float M = -INFINITY, L = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
+        float mc[4], lc[4];
+        float4 oc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + u;
+          mc[u] = c <= last ? __ldcg(&base[c].m[h]) : -INFINITY;
+          lc[u] = c <= last ? __ldcg(&base[c].l[h]) : 0.f;
+          oc[u] = c <= last ? __ldcg(reinterpret_cast<const float4*>(&base[c].O[h][4 * d4]))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (c0 + u <= last) merge_into(M, L, O, mc[u], lc[u], oc[u]);
+      }
+      store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, 1.f / L);
+    }
+    if (tid == 0) a.cnt[i] = 0;   // ready for the next launch (stream order)
   }
 
   // Drain: copies issued but not consumed (only after an abort) must land before exit.
@@ -774,8 +866,8 @@ cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t s
   a.sl2e = scale * kLog2e;
   a.spw = plan.spw;
   a.S = dv.S;
-  reinterpret_cast<KernelFn>(plan.fn)<<<plan.grid, plan.threads, plan.smem, st>>>(a, plan.tmap);
-  return cudaGetLastError();
+  return launch_dependent(reinterpret_cast<KernelFn>(plan.fn), dim3(plan.grid), dim3(plan.threads), plan.smem, st,
+                          a, plan.tmap);
 }
 
 }  // namespace dms
