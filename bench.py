@@ -183,6 +183,24 @@ def profile_traffic(workload: str, kernel: str):
     return None
 
 
+def rank_sequences(rank: int, batch: int) -> list[int]:
+    """Global sequence ids of one rank: every rank owns a full batch of its own (weak scaling)."""
+    return [rank * batch + b for b in range(batch)]
+
+
+def reduce_over_ranks(t_ms: float, nbytes: float, world: int, device) -> tuple[float, float]:
+    """(max over ranks of the timed region, sum over ranks of the bytes); identity at world == 1."""
+    if world <= 1:
+        return t_ms, nbytes
+    import torch
+    import torch.distributed as dist
+    v = torch.tensor([t_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(v, op=dist.ReduceOp.MAX)
+    b = torch.tensor([nbytes], dtype=torch.float64, device=device)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return float(v.item()), float(b.item())
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -252,7 +270,9 @@ def run_reference(args, wl, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name},
+        "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "q_heads": wl.num_q_heads,
+                   "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "window": wl.window,
+                   "context": wl.context if wl.ctx_range is None else list(wl.ctx_range)},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -281,12 +301,12 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     # this rank's sequences (weak scaling: every rank runs a full batch of its own sequences)
-    seqs = [rank * wl.batch + b for b in range(wl.batch)]
+    seqs = rank_sequences(rank, wl.batch)
     ctx_all = W.contexts(wl)
     ctx = np.array([ctx_all[b % wl.batch] for b in seqs])
     B, hkv, hq, d = wl.batch, wl.num_kv_heads, wl.num_q_heads, wl.head_dim
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    n_dec = args.warmup + args.steps * (1 if args.no_e2e else 2)
+    n_dec = args.warmup + args.steps * (2 if args.no_e2e else 3)   # timed, per-launch and e2e passes
     mps = int((ctx.max() + n_dec) // 16 + 2)
     scale = 1.0 / math.sqrt(d)
 
@@ -340,6 +360,7 @@ def main():
     launches0 = sum(c.launches() for c in caches)
     ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(args.steps * L)]
+    t_pl = args.warmup + args.steps   # first step of the per-launch pass
 
     def step(t, timed):
         for l in range(L):
@@ -348,7 +369,7 @@ def main():
             if l == 0:   # every layer holds the same tokens: one stats call gives the bytes of all
                 rc |= lib.dms_stats(h, sp, None, None, None, pT + t * 16)
             if timed:
-                e0, e1 = ev_pairs[(t - args.warmup) * L + l]
+                e0, e1 = ev_pairs[(t - t_pl) * L + l]
                 e0.record(stream)
             rc |= lib.dms_decode_attention(h, sp, B, pids, pQ + t * row_q, hq, scale, outs[l].data_ptr(),
                                            0 if tdt == torch.bfloat16 else 1)
@@ -366,13 +387,21 @@ def main():
     with ClockSampler(local) as clk:
         ev_start.record(stream)
         for t in range(args.warmup, args.warmup + args.steps):
-            step(t, True)
+            step(t, False)
         ev_end.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     t_ms = ev_start.elapsed_time(ev_end)
     launches = sum(c.launches() for c in caches) - launches0
+
+    # Per-launch pass: the next `steps` steps again, with an event pair around
+    # every attention launch. The events serialise each launch behind the one
+    # before it, so these durations include the launch latency that the
+    # timed region overlaps; they are the conservative per-kernel figure.
+    for t in range(t_pl, t_pl + args.steps):
+        step(t, True)
+    torch.cuda.synchronize()
     tot = totals.cpu().numpy()
     timed_tot = tot[args.warmup:args.warmup + args.steps]           # [steps, 2]
     bytes_launch = np.repeat(timed_tot[:, 1:2].astype(np.float64), L, axis=1) * d * 2 * wl.elem_bytes
@@ -381,64 +410,71 @@ def main():
     if any(x != same[0] for x in same):
         raise RuntimeError(f"layer caches diverged: {same}")
     attn_ms = np.array([a.elapsed_time(b) for a, b in ev_pairs])
+    pl_tot = tot[t_pl:t_pl + args.steps]
+    bytes_pl = np.repeat(pl_tot[:, 1:2].astype(np.float64), L, axis=1) * d * 2 * wl.elem_bytes
     status = [c.status() for c in caches]
     if any(status):
         raise RuntimeError(f"device status {status}")
 
     # max over ranks of the timed region; whole-job bytes
-    t_max_ms, bytes_all = t_ms, total_bytes
-    if world > 1:
-        v = torch.tensor([t_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(v, op=dist.ReduceOp.MAX)
-        t_max_ms = float(v.item())
-        v = torch.tensor([total_bytes], dtype=torch.float64, device=dev)
-        dist.all_reduce(v, op=dist.ReduceOp.SUM)
-        bytes_all = float(v.item())
+    t_max_ms, bytes_all = reduce_over_ranks(t_ms, total_bytes, world, dev)
     value = bytes_all / (t_max_ms * 1e-3) / 1e9
 
-    achieved = float(bytes_launch.mean()) / (float(attn_ms.mean()) * 1e-3) / 1e9
+    achieved = float(bytes_pl.mean()) / (float(attn_ms.mean()) * 1e-3) / 1e9
+
+    # Same kernel, L launches back to back between one event pair: no event
+    # between launches, so the launch latency the event pairs expose overlaps
+    # the previous launch (programmatic dependent launch). Reported beside the
+    # per-launch figure, not instead of it.
+    t_last = t_pl + args.steps - 1
+    burst_reps = 5
+    e_b0, e_b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_b0.record(stream)
+    for _ in range(burst_reps):
+        for l in range(L):
+            lib.dms_decode_attention(hs[l], sp, B, pids, pQ + t_last * row_q, hq, scale, outs[l].data_ptr(),
+                                     0 if tdt == torch.bfloat16 else 1)
+    e_b1.record(stream)
+    torch.cuda.synchronize()
+    burst_ms = e_b0.elapsed_time(e_b1) / (burst_reps * L)
+    achieved_burst = float(pl_tot[-1, 1]) * d * 2 * wl.elem_bytes / (burst_ms * 1e-3) / 1e9
     peak, peak_kind = peaks()
     kernel = {"auto": "mma" if tdt == torch.bfloat16 else "simt"}.get(args.attn_kernel, args.attn_kernel)
 
-    # ---- end-to-end pass through the public API with pinned host buffers
+    # ---- end-to-end pass through the public API with pinned host buffers: per
+    # step one host-to-device copy of each input (every layer appends the same
+    # new token rows) and one device-to-host copy of every layer's output
     e2e = None
     if not args.no_e2e:
         hK, hV, hA, hQ = (to_torch(x, None).pin_memory() for x in (Kd, Vd, Ad, Qd))
-        h_out = [torch.empty((B, hq, d), dtype=tdt).pin_memory() for _ in range(L)]
-        stage = [(torch.empty((B, hkv, d), dtype=tdt, device=dev), torch.empty((B, hkv, d), dtype=tdt, device=dev),
-                  torch.empty((B, hkv), dtype=torch.uint8, device=dev), torch.empty((B, hq, d), dtype=tdt, device=dev))
-                 for _ in range(L)]
-        t0_e2e = args.warmup + args.steps
+        h_out = torch.empty((L, B, hq, d), dtype=tdt).pin_memory()
+        d_out = torch.empty((L, B, hq, d), dtype=tdt, device=dev)
+        k_, v_ = torch.empty((B, hkv, d), dtype=tdt, device=dev), torch.empty((B, hkv, d), dtype=tdt, device=dev)
+        a_, q_ = torch.empty((B, hkv), dtype=torch.uint8, device=dev), torch.empty((B, hq, d), dtype=tdt, device=dev)
+        t0_e2e = t_pl + args.steps
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e_a.record(stream)
         for t in range(t0_e2e, t0_e2e + args.steps):
+            k_.copy_(hK[t], non_blocking=True)
+            v_.copy_(hV[t], non_blocking=True)
+            a_.copy_(hA[t], non_blocking=True)
+            q_.copy_(hQ[t], non_blocking=True)
             for l in range(L):
-                k_, v_, a_, q_ = stage[l]
-                k_.copy_(hK[t], non_blocking=True)
-                v_.copy_(hV[t], non_blocking=True)
-                a_.copy_(hA[t], non_blocking=True)
-                q_.copy_(hQ[t], non_blocking=True)
                 caches[l].append(ids, k_, v_, a_)
                 if l == 0:
                     lib.dms_stats(hs[l], sp, None, None, None, pT + t * 16)
-                caches[l].decode_attention(ids, q_, scale=scale, out=outs[l])
-                h_out[l].copy_(outs[l], non_blocking=True)
+                caches[l].decode_attention(ids, q_, scale=scale, out=d_out[l])
+            h_out.copy_(d_out, non_blocking=True)
         e_b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e_a.elapsed_time(e_b)
         tot2 = totals.cpu().numpy()[t0_e2e:t0_e2e + args.steps]
         e2e_bytes = float(tot2[:, 1].astype(np.float64).sum()) * L * d * 2 * wl.elem_bytes
-        if world > 1:
-            v = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(v, op=dist.ReduceOp.MAX)
-            e2e_ms = float(v.item())
-            v = torch.tensor([e2e_bytes], dtype=torch.float64, device=dev)
-            dist.all_reduce(v, op=dist.ReduceOp.SUM)
-            e2e_bytes = float(v.item())
-        h2d = L * (2 * row_kv + B * hkv + row_q)
+        e2e_ms, e2e_bytes = reduce_over_ranks(e2e_ms, e2e_bytes, world, dev)
+        h2d = 2 * row_kv + B * hkv + row_q
         d2h = L * B * hq * d * wl.elem_bytes
         e2e = {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
@@ -479,7 +515,11 @@ def main():
                          "kernel": f"dms_decode_attention ({kernel})",
                          "launch_ms_mean": float(attn_ms.mean()), "launch_ms_p10": float(np.percentile(attn_ms, 10)),
                          "launch_ms_p90": float(np.percentile(attn_ms, 90)),
-                         "bytes_per_launch": float(bytes_launch.mean())},
+                         "bytes_per_launch": float(bytes_pl.mean()),
+                         "launch_timing": "CUDA event pair around every launch, in a second pass over the "
+                                          "next steps; burst: L launches between one event pair",
+                         "launch_ms_burst": burst_ms, "achieved_burst": achieved_burst,
+                         "frac_burst": achieved_burst / peak},
             "gpu_launches": launches,
             "clocks": clk.summary(),
         }
