@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--workload", default="qwen-r1-7b-32k", choices=sorted(W.WORKLOADS))
     ap.add_argument("--layers", type=int, default=0, help="layer caches per step (0: enough to exceed 8x L2)")
     ap.add_argument("--attn-kernel", default="auto", choices=["auto", "mma", "simt"])
+    ap.add_argument("--step", default="fused", choices=["fused", "separate"],
+                    help="fused: one dms_decode_step launch per layer; separate: dms_append + dms_decode_attention")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -166,10 +168,10 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profile_traffic(workload: str, kernel: str):
-    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary,
+def profile_traffic(workload: str, kernel: str, entry: str = "dms_decode_attention"):
+    """Per-launch DRAM bytes of the timed kernel from the committed ncu summary,
     valid only while the kernel source is unchanged since the capture."""
-    path = os.path.join(ROOT, "profiles", f"dms_decode_attention_{kernel}_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{entry}_{kernel}_{workload}.md")
     src = os.path.join(ROOT, "learned_kv_cache_decode_b200", "csrc", "dms_attention.cu")
     try:
         text = open(path).read()
@@ -306,7 +308,9 @@ def main():
     ctx = np.array([ctx_all[b % wl.batch] for b in seqs])
     B, hkv, hq, d = wl.batch, wl.num_kv_heads, wl.num_q_heads, wl.head_dim
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    n_dec = args.warmup + args.steps * (2 if args.no_e2e else 3)   # timed, per-launch and e2e passes
+    burst_steps = 5
+    # timed, per-launch, burst and e2e passes
+    n_dec = args.warmup + args.steps * (2 if args.no_e2e else 3) + burst_steps
     mps = int((ctx.max() + n_dec) // 16 + 2)
     scale = 1.0 / math.sqrt(d)
 
@@ -362,19 +366,27 @@ def main():
                 for _ in range(args.steps * L)]
     t_pl = args.warmup + args.steps   # first step of the per-launch pass
 
+    fused = args.step == "fused"
+    odt = 0 if tdt == torch.bfloat16 else 1
+
     def step(t, timed):
         for l in range(L):
             h = hs[l]
-            rc = lib.dms_append(h, sp, B, pids, None, B, pK + t * row_kv, pV + t * row_kv, pA + t * B * hkv)
-            if l == 0:   # every layer holds the same tokens: one stats call gives the bytes of all
-                rc |= lib.dms_stats(h, sp, None, None, None, pT + t * 16)
+            rc = 0
+            if not fused:
+                rc |= lib.dms_append(h, sp, B, pids, None, B, pK + t * row_kv, pV + t * row_kv, pA + t * B * hkv)
             if timed:
                 e0, e1 = ev_pairs[(t - t_pl) * L + l]
                 e0.record(stream)
-            rc |= lib.dms_decode_attention(h, sp, B, pids, pQ + t * row_q, hq, scale, outs[l].data_ptr(),
-                                           0 if tdt == torch.bfloat16 else 1)
+            if fused:
+                rc |= lib.dms_decode_step(h, sp, B, pids, pK + t * row_kv, pV + t * row_kv, pA + t * B * hkv,
+                                          pQ + t * row_q, hq, scale, outs[l].data_ptr(), odt)
+            else:
+                rc |= lib.dms_decode_attention(h, sp, B, pids, pQ + t * row_q, hq, scale, outs[l].data_ptr(), odt)
             if timed:
                 e1.record(stream)
+            if l == 0:   # every layer holds the same tokens: one stats call gives the bytes of all
+                rc |= lib.dms_stats(h, sp, None, None, None, pT + t * 16)
             if rc:
                 raise RuntimeError(f"library call failed ({rc})")
 
@@ -422,22 +434,31 @@ def main():
 
     achieved = float(bytes_pl.mean()) / (float(attn_ms.mean()) * 1e-3) / 1e9
 
-    # Same kernel, L launches back to back between one event pair: no event
-    # between launches, so the launch latency the event pairs expose overlaps
-    # the previous launch (programmatic dependent launch). Reported beside the
-    # per-launch figure, not instead of it.
-    t_last = t_pl + args.steps - 1
-    burst_reps = 5
+    # Burst: `burst_steps` more steps between one event pair, no event between
+    # launches, so each launch's set-up overlaps the launch before it
+    # (programmatic dependent launch). Separate mode times the attention
+    # launches alone. Reported beside the per-launch figure, not instead of it.
+    t_b = t_pl + args.steps
     e_b0, e_b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_b0.record(stream)
-    for _ in range(burst_reps):
-        for l in range(L):
-            lib.dms_decode_attention(hs[l], sp, B, pids, pQ + t_last * row_q, hq, scale, outs[l].data_ptr(),
-                                     0 if tdt == torch.bfloat16 else 1)
-    e_b1.record(stream)
+    if fused:
+        e_b0.record(stream)
+        for t in range(t_b, t_b + burst_steps):
+            step(t, False)
+        e_b1.record(stream)
+    else:
+        for t in range(t_b, t_b + burst_steps):   # keep the decode going: append outside the events
+            for l in range(L):
+                lib.dms_append(hs[l], sp, B, pids, None, B, pK + t * row_kv, pV + t * row_kv, pA + t * B * hkv)
+            lib.dms_stats(hs[0], sp, None, None, None, pT + t * 16)
+        e_b0.record(stream)
+        for t in range(t_b, t_b + burst_steps):
+            for l in range(L):
+                lib.dms_decode_attention(hs[l], sp, B, pids, pQ + t * row_q, hq, scale, outs[l].data_ptr(), odt)
+        e_b1.record(stream)
     torch.cuda.synchronize()
-    burst_ms = e_b0.elapsed_time(e_b1) / (burst_reps * L)
-    achieved_burst = float(pl_tot[-1, 1]) * d * 2 * wl.elem_bytes / (burst_ms * 1e-3) / 1e9
+    burst_ms = e_b0.elapsed_time(e_b1) / (burst_steps * L)
+    b_tot = totals.cpu().numpy()[t_b:t_b + burst_steps]
+    achieved_burst = float(b_tot[:, 1].astype(np.float64).mean()) * d * 2 * wl.elem_bytes / (burst_ms * 1e-3) / 1e9
     peak, peak_kind = peaks()
     kernel = {"auto": "mma" if tdt == torch.bfloat16 else "simt"}.get(args.attn_kernel, args.attn_kernel)
 
@@ -451,7 +472,7 @@ def main():
         d_out = torch.empty((L, B, hq, d), dtype=tdt, device=dev)
         k_, v_ = torch.empty((B, hkv, d), dtype=tdt, device=dev), torch.empty((B, hkv, d), dtype=tdt, device=dev)
         a_, q_ = torch.empty((B, hkv), dtype=torch.uint8, device=dev), torch.empty((B, hq, d), dtype=tdt, device=dev)
-        t0_e2e = t_pl + args.steps
+        t0_e2e = t_b + burst_steps
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -463,10 +484,13 @@ def main():
             a_.copy_(hA[t], non_blocking=True)
             q_.copy_(hQ[t], non_blocking=True)
             for l in range(L):
-                caches[l].append(ids, k_, v_, a_)
+                if fused:
+                    caches[l].decode_step(ids, k_, v_, a_, q_, scale=scale, out=d_out[l])
+                else:
+                    caches[l].append(ids, k_, v_, a_)
+                    caches[l].decode_attention(ids, q_, scale=scale, out=d_out[l])
                 if l == 0:
                     lib.dms_stats(hs[l], sp, None, None, None, pT + t * 16)
-                caches[l].decode_attention(ids, q_, scale=scale, out=d_out[l])
             h_out.copy_(d_out, non_blocking=True)
         e_b.record(stream)
         torch.cuda.synchronize()
@@ -504,15 +528,18 @@ def main():
                 "layers": L, "attn_kernel": kernel, "parallelism": f"replicas x{world}",
                 "l2": f"inputs larger than L2: {L} layer pools, {layer_bytes / 2**20:.0f} MiB retained K/V each "
                       f"({L * layer_bytes / 2**20:.0f} MiB per step vs 126 MiB L2)",
-                "step": "per layer: dms_append (1 token/seq) + dms_decode_attention; one dms_stats per step",
+                "step": ("per layer: dms_decode_step (append 1 token/seq + attention, one launch)" if fused else
+                         "per layer: dms_append (1 token/seq) + dms_decode_attention") + "; one dms_stats per step",
             },
             "decode_steps_per_s_per_layer": n_layer_steps / (t_max_ms * 1e-3),
             "retained_bytes_per_step": total_bytes / args.steps,
             "compression_ratio": float(timed_tot[-1, 0] / timed_tot[-1, 1]),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": profile_traffic(wl.name, kernel),
-                         "kernel": f"dms_decode_attention ({kernel})",
+                         "traffic": profile_traffic(wl.name, kernel,
+                                                    "dms_decode_step" if fused else "dms_decode_attention"),
+                         "kernel": f"dms_decode_step ({kernel}, append fused)" if fused else
+                                   f"dms_decode_attention ({kernel})",
                          "launch_ms_mean": float(attn_ms.mean()), "launch_ms_p10": float(np.percentile(attn_ms, 10)),
                          "launch_ms_p90": float(np.percentile(attn_ms, 90)),
                          "bytes_per_launch": float(bytes_pl.mean()),

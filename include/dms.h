@@ -145,6 +145,28 @@ dms_status dms_decode_attention(dms_cache* cache, cudaStream_t stream, int32_t n
                                 const int32_t* seq_ids, const void* Q, int32_t num_q_heads,
                                 float scale, void* out, dms_dtype out_dtype);
 
+/* One whole decode step in one launch: dms_append of one token per sequence
+ * (cu_tokens = NULL) followed by dms_decode_attention, with the same results:
+ * the same bookkeeping bit for bit, and outputs equal up to fp32 rounding
+ * order (scope row "fused append + attention", paper summary, Key claims:
+ * decode is bound by memory reads, so the step should cost one pass over
+ * the retained K/V and one launch).
+ * The attention runs over the cache as it was before the step, with the row
+ * of the token that leaves at this step masked and the new token taken
+ * from K and V; the append's writes go to rows that no part of the launch
+ * attends. A cache with more than 1024 streams (max_seqs * num_kv_heads), or
+ * whose configuration leaves no shared memory for the step's per-stream
+ * state, issues the two launches instead.
+ *   n_seqs, seq_ids      as dms_append (one token per sequence)
+ *   K, V                 device [n_seqs, num_kv_heads, head_dim] of the cache dtype, 16-B aligned
+ *   alpha                device uint8 [n_seqs, num_kv_heads]
+ *   Q, num_q_heads, scale, out, out_dtype   as dms_decode_attention
+ * Device errors latch as in dms_append (pool exhausted, stream full, bad
+ * seq id); the outputs of that launch are then unspecified. Async. */
+dms_status dms_decode_step(dms_cache* cache, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                           const void* K, const void* V, const uint8_t* alpha, const void* Q,
+                           int32_t num_q_heads, float scale, void* out, dms_dtype out_dtype);
+
 /* Retained counts and compression ratios (paper summary, Key claims: CR =
  * tokens seen / tokens kept; each head can land at its own CR). Async;
  * every output is device memory and optional (NULL skips it).

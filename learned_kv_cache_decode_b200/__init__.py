@@ -107,6 +107,21 @@ class DmsCache:
                                                     _DTYPES[out.dtype]), "dms_decode_attention")
         return out
 
+    def decode_step(self, seq_ids: torch.Tensor, K: torch.Tensor, V: torch.Tensor, alpha: torch.Tensor,
+                    Q: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None,
+                    out_dtype: torch.dtype | None = None) -> torch.Tensor:
+        """One decode step in one launch: append one token per sequence (K, V [B, Hkv, d],
+        alpha uint8 [B, Hkv]) and attend with Q [B, Hq, d] -> out [B, Hq, d]."""
+        b, hq, d = Q.shape
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        if out is None:
+            out = torch.empty((b, hq, d), dtype=out_dtype or Q.dtype, device=Q.device)
+        _native.check(self.lib.dms_decode_step(self._h, _stream(), int(seq_ids.numel()), _ptr(seq_ids), _ptr(K),
+                                               _ptr(V), _ptr(alpha), _ptr(Q), hq, float(scale), _ptr(out),
+                                               _DTYPES[out.dtype]), "dms_decode_step")
+        return out
+
     # -- inspection --------------------------------------------------------
     def stats(self) -> dict:
         """Device tensors: retained [S], seen [S], head_cr [Hkv], totals [2] (async)."""

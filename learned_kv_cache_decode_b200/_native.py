@@ -29,7 +29,7 @@ DMS_ATTN_MMA = 2
 
 EXPORTS = ("dms_cache_create", "dms_cache_destroy", "dms_cache_reset", "dms_seq_reset", "dms_append",
            "dms_decode_attention", "dms_stats", "dms_snapshot", "dms_gather_kv", "dms_get_status",
-           "dms_status_string", "dms_launch_count", "dms_decode_attention_noalloc")
+           "dms_status_string", "dms_launch_count", "dms_decode_attention_noalloc", "dms_decode_step")
 
 DMS_NOALLOC_MAX_STREAMS = 512
 DMS_NOALLOC_MAX_PIECES = 1024
@@ -109,6 +109,8 @@ def load() -> ctypes.CDLL:
     L.dms_status_string.restype = ctypes.c_char_p
     L.dms_launch_count.argtypes = [p]
     L.dms_launch_count.restype = i64
+    L.dms_decode_step.argtypes = [p, p, i32, p, p, p, p, p, i32, ctypes.c_float, p, ctypes.c_int]
+    L.dms_decode_step.restype = st
     L.dms_decode_attention_noalloc.argtypes = [p, ctypes.POINTER(DmsPagedKv), i32, p, p, i32, ctypes.c_float, p,
                                                ctypes.c_int]
     L.dms_decode_attention_noalloc.restype = st

@@ -15,6 +15,8 @@ struct dms_cache {
   int num_sms = 0;
   dms::Dev dv{};
   dms::AttnPlan plan{};
+  dms::AttnPlan step_plan{};   // fused decode step (append + attention in one launch)
+  bool has_step = false;       // else dms_decode_step issues the two launches
   int64_t launches = 0;
   bool poisoned = false;   // a device error was observed by dms_get_status
 };
@@ -105,8 +107,14 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
   step(alloc(&dv.kv, (size_t)dv.max_pages * 2 * dms::kPage * dv.d * dv.elem_bytes));
   if (e == cudaSuccess) e = dms::prepare_aux_kernels();
   if (e == cudaSuccess) e = dms::attention_prepare(dv, c.dtype, c.attn_kernel, h->num_sms, &h->plan);
-  if (e == cudaSuccess)
-    e = alloc(&dv.part, ((size_t)h->plan.grid + dv.S) * dms::kMaxGroup * (dv.d + 2));
+  if (e == cudaSuccess && dv.S <= dms::kStepMaxStreams) {
+    // The fused step needs its per-stream decisions in shared memory; a
+    // configuration that leaves no room for them falls back to two launches.
+    h->has_step = dms::step_prepare(dv, c.dtype, c.attn_kernel, h->num_sms, &h->step_plan) == cudaSuccess;
+    cudaGetLastError();
+  }
+  const int grid = h->has_step && h->step_plan.grid > h->plan.grid ? h->step_plan.grid : h->plan.grid;
+  if (e == cudaSuccess) e = alloc(&dv.part, ((size_t)grid + dv.S) * dms::kMaxGroup * (dv.d + 2));
   if (e == cudaSuccess) e = cudaMemset(dv.kv, 0, (size_t)dv.max_pages * 2 * dms::kPage * dv.d * dv.elem_bytes);
   if (e == cudaSuccess) e = cudaMemset(dv.page_table, 0xff, S * dv.mps * sizeof(int32_t));
   if (e == cudaSuccess) e = cudaMemset(dv.slot_pos, 0xff, (size_t)dv.max_pages * dms::kPage * sizeof(int32_t));
@@ -186,6 +194,31 @@ dms_status dms_decode_attention(dms_cache* h, cudaStream_t stream, int32_t n_seq
   h->launches += 1;
   return from_cuda(dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
                                          out_dtype == DMS_F32));
+}
+
+dms_status dms_decode_step(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                           const void* K, const void* V, const uint8_t* alpha, const void* Q, int32_t num_q_heads,
+                           float scale, void* out, dms_dtype out_dtype) {
+  if (!h || n_seqs < 0 || n_seqs > h->cfg.max_seqs) return DMS_ERR_INVALID;
+  if (dms_status s = check_usable(h)) return s;
+  if (num_q_heads < h->cfg.num_kv_heads || num_q_heads % h->cfg.num_kv_heads != 0) return DMS_ERR_INVALID;
+  if (num_q_heads / h->cfg.num_kv_heads > dms::kMaxGroup) return DMS_ERR_INVALID;
+  if (out_dtype != DMS_BF16 && out_dtype != DMS_F32) return DMS_ERR_INVALID;
+  if (n_seqs == 0) return DMS_OK;
+  if (!seq_ids || !K || !V || !alpha || !Q || !out) return DMS_ERR_INVALID;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(out)) return DMS_ERR_INVALID;
+  if (!h->has_step) {
+    int launches = 0;
+    cudaError_t e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, &launches);
+    h->launches += launches;
+    if (e != cudaSuccess) return DMS_ERR_CUDA;
+    h->launches += 1;
+    return from_cuda(dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
+                                           out_dtype == DMS_F32));
+  }
+  h->launches += 1;
+  return from_cuda(dms::launch_step(h->dv, h->step_plan, stream, n_seqs, seq_ids, K, V, alpha, Q, num_q_heads,
+                                    scale, out, out_dtype == DMS_F32));
 }
 
 dms_status dms_stats(dms_cache* h, cudaStream_t stream, int32_t* retained, int32_t* seen, float* head_cr,

@@ -44,6 +44,15 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// A decode step fused into the attention launch: the new token of every call
+// stream and the cache the append writes.
+struct StepArgs {
+  const uint8_t* K;       // [n_seqs][hkv][d] new key rows
+  const uint8_t* V;       // [n_seqs][hkv][d] new value rows
+  const uint8_t* alpha;   // [n_seqs][hkv] eviction decisions of the new tokens
+  Dev dv;                 // the cache, writable
+};
+
 struct AttnArgs {
   const int32_t* seq_ids;
   const uint8_t* Q;
@@ -58,6 +67,7 @@ struct AttnArgs {
   float sl2e;   // softmax scale * log2(e): scores live in the base-2 domain
   int spw;      // TMA stages per warp
   int S;        // streams of the cache (sizes the plan arrays in shared memory)
+  StepArgs step;   // used by the fused decode-step kernel only
 };
 
 // Largest i in [0, n] with prefix[i] <= x (prefix is non-decreasing, prefix[0] = 0).
@@ -156,10 +166,12 @@ struct MmaOffsets {
 };
 
 // NP pages of one stream at once: their QK products, one shared online-
-// softmax update, then their PV products. `valid[p]` tokens of page p are
+// softmax update, then their PV products. Bit r of `rows[p]` says whether
+// row r of page p is a token to attend (all 16 except in a stream's last
+// page, or where a leaving token's row is masked); the others are
 // real (16 except in a stream's last page).
 template <int D, int NP>
-__device__ __forceinline__ void mma_pages(MmaState<D>& S, const uint32_t (&stage)[NP], const int (&valid)[NP],
+__device__ __forceinline__ void mma_pages(MmaState<D>& S, const uint32_t (&stage)[NP], const uint32_t (&rows)[NP],
                                           float sl2e, int lane, const MmaOffsets<D>& off) {
   // ---- S^T = K * Q^T per page: rows = 16 tokens, cols = 8 heads
   float v[NP][4];
@@ -179,9 +191,9 @@ __device__ __forceinline__ void mma_pages(MmaState<D>& S, const uint32_t (&stage
   const int t0 = lane >> 2;
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
-    if (valid[p] < kPage) {
-      if (t0 >= valid[p])     { v[p][0] = -INFINITY; v[p][1] = -INFINITY; }
-      if (t0 + 8 >= valid[p]) { v[p][2] = -INFINITY; v[p][3] = -INFINITY; }
+    if (rows[p] != 0xffffu) {
+      if (!((rows[p] >> t0) & 1u))       { v[p][0] = -INFINITY; v[p][1] = -INFINITY; }
+      if (!((rows[p] >> (t0 + 8)) & 1u)) { v[p][2] = -INFINITY; v[p][3] = -INFINITY; }
     }
   }
   // ---- online softmax per head column (tokens spread over lanes with equal lane % 4)
@@ -197,19 +209,24 @@ __device__ __forceinline__ void mma_pages(MmaState<D>& S, const uint32_t (&stage
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
   }
   const float mn0 = fmaxf(S.m[0], mx0), mn1 = fmaxf(S.m[1], mx1);
+  // While every row seen so far is masked the max is -inf; exponents then
+  // use 0 as the reference, so that masked rows give 0, not -inf - -inf.
+  const float ref0 = mn0 == -INFINITY ? 0.f : mn0, ref1 = mn1 == -INFINITY ? 0.f : mn1;
   float pr[NP][4];
   float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
-    pr[p][0] = ex2(v[p][0] - mn0);
-    pr[p][1] = ex2(v[p][1] - mn1);
-    pr[p][2] = ex2(v[p][2] - mn0);
-    pr[p][3] = ex2(v[p][3] - mn1);
+    pr[p][0] = ex2(v[p][0] - ref0);
+    pr[p][1] = ex2(v[p][1] - ref1);
+    pr[p][2] = ex2(v[p][2] - ref0);
+    pr[p][3] = ex2(v[p][3] - ref1);
     sum0 += pr[p][0] + pr[p][2];
     sum1 += pr[p][1] + pr[p][3];
   }
   if (__any_sync(0xffffffffu, (mn0 != S.m[0]) | (mn1 != S.m[1]))) {   // the running max moved
-    const float c0 = ex2(S.m[0] - mn0), c1 = ex2(S.m[1] - mn1);
+    // a column that has seen nothing (m = -inf) holds l = 0 and O = 0: factor 0
+    const float c0 = S.m[0] == -INFINITY ? 0.f : ex2(S.m[0] - mn0);
+    const float c1 = S.m[1] == -INFINITY ? 0.f : ex2(S.m[1] - mn1);
     S.l[0] *= c0;
     S.l[1] *= c1;
 #pragma unroll
@@ -231,9 +248,9 @@ __device__ __forceinline__ void mma_pages(MmaState<D>& S, const uint32_t (&stage
     const uint32_t pb0 = movmatrix_trans(pack_bf16x2(pr[p][0], pr[p][1]));   // tokens 0..7
     const uint32_t pb1 = movmatrix_trans(pack_bf16x2(pr[p][2], pr[p][3]));   // tokens 8..15
     uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
-    if (valid[p] < kPage) {   // rows past n may hold stale bits: zero them
-      keep0 = (tk < valid[p] ? 0x0000ffffu : 0u) | (tk + 1 < valid[p] ? 0xffff0000u : 0u);
-      keep1 = (tk + 8 < valid[p] ? 0x0000ffffu : 0u) | (tk + 9 < valid[p] ? 0xffff0000u : 0u);
+    if (rows[p] != 0xffffu) {   // masked rows may hold stale bits: zero them
+      keep0 = (((rows[p] >> tk) & 1u) ? 0x0000ffffu : 0u) | (((rows[p] >> (tk + 1)) & 1u) ? 0xffff0000u : 0u);
+      keep1 = (((rows[p] >> (tk + 8)) & 1u) ? 0x0000ffffu : 0u) | (((rows[p] >> (tk + 9)) & 1u) ? 0xffff0000u : 0u);
     }
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
@@ -330,8 +347,10 @@ __device__ __forceinline__ void simt_start(SimtState<D>& S, const SimtQuery<D>& 
 }
 
 template <int D, typename E>
-__device__ __forceinline__ void simt_page(SimtState<D>& S, const E* stage, int valid, int g, int lane) {
-  for (int t = 0; t < valid; ++t) {
+__device__ __forceinline__ void simt_page(SimtState<D>& S, const E* stage, uint32_t rows, int g, int lane) {
+  const int end = 32 - __clz(rows);   // one past the highest row to attend
+  for (int t = 0; t < end; ++t) {
+    if (!((rows >> t) & 1u)) continue;
     float k[D / 32], v[D / 32];
     simt_load_row<D, E>(stage + (size_t)t * D, lane, k);
     simt_load_row<D, E>(stage + (size_t)(kPage + t) * D, lane, v);
@@ -392,9 +411,16 @@ __device__ __forceinline__ void store_out4(const AttnArgs& a, int b, int h, int 
   }
 }
 
-// Online merge of partial (m2, l2, o2) into (m, l, o); scores in base 2.
-// At least one of m, m2 must be finite.
+// Online merge of partial (m2, l2, o2) into (m, l, o); scores in base 2. A
+// side with m = -inf saw no token and contributes nothing.
 __device__ __forceinline__ void merge_into(float& m, float& l, float4& o, float m2, float l2, float4 o2) {
+  if (m2 == -INFINITY) return;   // the other side saw nothing
+  if (m == -INFINITY) {          // this side saw nothing
+    m = m2;
+    l = l2;
+    o = o2;
+    return;
+  }
   const float mn = fmaxf(m, m2);
   const float sa = ex2(m - mn), sb = ex2(m2 - mn);   // 0 for a side that saw nothing (m = -inf)
   l = l * sa + l2 * sb;
@@ -405,20 +431,234 @@ __device__ __forceinline__ void merge_into(float& m, float& l, float4& o, float 
   m = mn;
 }
 
+// Four consecutive elements of a row as floats (p 8-byte aligned for bf16,
+// 16-byte aligned for f32).
+template <typename E>
+__device__ __forceinline__ void load4(const E* p, float (&x)[4]);
+template <>
+__device__ __forceinline__ void load4<float>(const float* p, float (&x)[4]) {
+  const float4 f = *reinterpret_cast<const float4*>(p);
+  x[0] = f.x;
+  x[1] = f.y;
+  x[2] = f.z;
+  x[3] = f.w;
+}
+template <>
+__device__ __forceinline__ void load4<uint16_t>(const uint16_t* p, float (&x)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  x[0] = bf16_lo(u.x);
+  x[1] = bf16_hi(u.x);
+  x[2] = bf16_lo(u.y);
+  x[3] = bf16_hi(u.y);
+}
+
+// The step's new token of call stream i, for query head h and dims
+// [4 d4, 4 d4 + 4): merged into (M, L, O) when `use`. Its score is q . k in
+// fp32 from the stored inputs, scaled into base 2 like the page scores.
+// Warp-collective: the D/4 lanes of one head reduce the dot product, so
+// every lane of the warp calls it, `use` or not.
+template <int D, typename E>
+__device__ __forceinline__ void add_new_token(const AttnArgs& a, int i, int h, int d4, bool use, float& M,
+                                              float& L, float4& O) {
+  const int b = i / a.hkv, kvh = i % a.hkv;
+  float q4[4], k4[4], v4[4];
+  load4<E>(reinterpret_cast<const E*>(a.Q) + ((size_t)b * a.hq + (size_t)kvh * a.g + h) * D + 4 * d4, q4);
+  load4<E>(reinterpret_cast<const E*>(a.step.K) + (size_t)i * D + 4 * d4, k4);
+  load4<E>(reinterpret_cast<const E*>(a.step.V) + (size_t)i * D + 4 * d4, v4);
+  float dot = q4[0] * k4[0] + q4[1] * k4[1] + q4[2] * k4[2] + q4[3] * k4[3];
+#pragma unroll
+  for (int o = D / 8; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  if (use) merge_into(M, L, O, dot * a.sl2e, 1.f, make_float4(v4[0], v4[1], v4[2], v4[3]));
+}
+
+// Combine the partials first .. last of stream i into its output, items
+// [t_begin, items) with stride t_step (a multiple of 32; every lane of a
+// calling warp runs the same iterations). The caller has acquired them.
+template <int D, typename E, bool STEP>
+__device__ __forceinline__ void combine_stream(const AttnArgs& a, int i, int first, int last, int t_begin,
+                                               int t_step, bool add_new) {
+  const int b = i / a.hkv, kvh = i % a.hkv;
+  const int items = a.g * (D / 4);
+  const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
+  for (int t0 = 0; t0 < items; t0 += t_step) {
+    const int t = t0 + t_begin;
+    const bool live = t < items;
+    if (!__any_sync(0xffffffffu, live)) break;   // warp-uniform
+    const int h = (live ? t : 0) / (D / 4), d4 = (live ? t : 0) % (D / 4);
+    float M = -INFINITY, L = 0.f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
+      float mc[4], lc[4];
+      float4 oc[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u;
+        mc[u] = c <= last ? __ldcg(&base[c].m[h]) : -INFINITY;
+        lc[u] = c <= last ? __ldcg(&base[c].l[h]) : 0.f;
+        oc[u] = c <= last ? __ldcg(reinterpret_cast<const float4*>(&base[c].O[h][4 * d4]))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + u <= last) merge_into(M, L, O, mc[u], lc[u], oc[u]);
+    }
+    if constexpr (STEP) add_new_token<D, E>(a, i, h, d4, add_new, M, L, O);   // warp-collective
+    if (live) store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, L > 0.f ? 1.f / L : 0.f);
+  }
+}
+
+// The step warp of a fused decode step (one warp per CTA).
+//  1. For every call stream, from the pre-step state read by the plan and the
+//     leaving slot the consumer warps read from the window ring: does the
+//     token at s - w leave now (its slot is reused), or does the new token
+//     take the fresh slot n (popping a page when n is a multiple of 16)? Pops are ranked in stream order (warp scan), exactly
+//     as dms_append ranks them; a pool too small for all pops fails every
+//     stream that needs one.
+//  2. Publishes the decisions to the CTA's consumers, then counts this CTA as
+//     having read the pre-step state.
+//  3. Writes the outputs of this CTA's streams that had nothing retained (the
+//     new token alone: its value row).
+//  4. Once every CTA has read the pre-step state, appends this CTA's streams
+//     (i = blockIdx.x mod gridDim.x): bookkeeping and K/V rows. CTA 0 latches
+//     the errors the plan found and moves the free stack.
+template <int D, typename E>
+__device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int* prefix, const int* sid,
+                                       const int* s_nold, const int* s_pos, int* s_rslot, int* s_tslot,
+                                       int* s_flag, int* s_rank, int* misc, bool healthy,
+                                       volatile int* abort_flag) {
+  const int lane = threadIdx.x & 31;
+  const Dev& dv = a.step.dv;
+  // Wait (no spinning) until the consumer warps have resolved every stream's
+  // leaving slot (s_rslot): they arrive at barrier 2 without waiting.
+  named_barrier(2, blockDim.x);
+  if (healthy) {
+    const int per = (nst + 31) / 32;   // contiguous streams per lane: the scan keeps stream order
+    const int b0 = min(lane * per, nst), e0 = min(b0 + per, nst);
+    int cnt = 0;
+    for (int i = b0; i < e0; ++i) {
+      int f = s_flag[i], ts = -1;
+      if (!(f & 4)) {
+        const int rs = s_rslot[i];   // token s - w leaves now and s takes its slot
+        ts = rs >= 0 ? rs : s_nold[i];
+        if (rs < 0 && (ts % kPage) == 0) {
+          if (ts / kPage >= dv.mps) {
+            f |= 8;
+            ts = -1;
+          } else {
+            f |= 1;
+            ++cnt;
+          }
+        }
+      }
+      s_tslot[i] = ts;
+      s_flag[i] = f;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    const int fc = misc[12];   // free-stack depth, read by the plan
+    const bool fits = total <= fc;
+    int rank = incl - cnt;
+    for (int i = b0; i < e0; ++i) {
+      if (!(s_flag[i] & 1)) continue;
+      if (fits) {
+        s_rank[i] = rank++;
+      } else {
+        s_tslot[i] = -1;   // pool exhausted: this stream is left unchanged
+        s_flag[i] |= 16;
+      }
+    }
+    if (lane == 0) misc[13] = fits ? total : -1;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence_block();
+    *reinterpret_cast<volatile int*>(&misc[15]) = 1;   // the consumers may read the decisions
+    // This CTA is done reading the pre-step state (its reads were ordered
+    // before this point by the plan's barriers and barrier 2).
+    red_add_release_gpu(&a.ctrl[kCtrlPlanned], 1);
+  }
+  __syncwarp();
+  if (!healthy) return;
+
+  const int G = gridDim.x;
+  // Streams with nothing retained before the step attend to the new token alone.
+  for (int i = blockIdx.x; i < nst; i += G) {
+    if (prefix[i + 1] != prefix[i]) continue;
+    const int b = i / a.hkv, kvh = i % a.hkv;
+    const bool app = s_tslot[i] >= 0;
+    for (int e = lane; e < a.g * (D / 4); e += 32) {
+      const int h = e / (D / 4), d4 = e % (D / 4);
+      float v4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (app) load4<E>(reinterpret_cast<const E*>(a.step.V) + (size_t)i * D + 4 * d4, v4);
+      store_out4(a, b, kvh * a.g + h, 4 * d4, D, make_float4(v4[0], v4[1], v4[2], v4[3]), 1.f);
+    }
+  }
+
+  // Wait until every CTA has read the pre-step state, then write the append.
+  if (lane == 0) {
+    wait_flag_ge(reinterpret_cast<volatile int*>(&a.ctrl[kCtrlPlanned]), G, abort_flag, a.ctrl, 200);
+    fence_acq_rel_gpu();   // acquire: every CTA's reads of the pre-step state happen before our writes
+  }
+  __syncwarp();
+  if (blockIdx.x == 0 && lane == 0) {
+    for (int i = 0; i < nst; ++i) {
+      const int f = s_flag[i];
+      if (f & 4) latch(a.ctrl, DMS_ERR_BAD_SEQ);
+      if (f & 8) latch(a.ctrl, DMS_ERR_STREAM_FULL);
+      if (f & 16) latch(a.ctrl, DMS_ERR_POOL_EXHAUSTED);
+    }
+    if (misc[13] > 0) dv.ctrl[kCtrlFree] = misc[12] - misc[13];
+  }
+  const int row_bytes = D * (int)sizeof(E);
+  const int vec = row_bytes / 16;
+  for (int i = blockIdx.x; i < nst; i += G) {
+    const int ts = s_tslot[i];
+    if (ts < 0) continue;
+    const int st = sid[i], s = s_pos[i], f = s_flag[i];
+    const int lp = ts / kPage;
+    const int page = (f & 1) ? dv.free_list[misc[12] - 1 - s_rank[i]] : dv.page_table[(size_t)st * dv.mps + lp];
+    if (page < 0 || page >= dv.max_pages) {
+      if (lane == 0) latch(a.ctrl, DMS_ERR_INVALID);
+      continue;
+    }
+    if (lane == 0) {
+      if (f & 1) {
+        dv.page_table[(size_t)st * dv.mps + lp] = page;
+        dv.n_pages[st] = lp + 1;
+      }
+      if (s_rslot[i] < 0) dv.n[st] = s_nold[i] + 1;
+      dv.ring[(size_t)st * dv.w + (s % dv.w)] = (ts << 1) | ((f >> 1) & 1);
+      dv.pos[st] = s + 1;
+      dv.slot_pos[(size_t)page * kPage + ts % kPage] = s;
+    }
+    for (int v = lane; v < 2 * vec; v += 32) {
+      const int which = v / vec, c = v % vec;
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>((which ? a.step.V : a.step.K) + (size_t)i * row_bytes) + c);
+      reinterpret_cast<uint4*>(dv.kv + ((size_t)page * 2 * kPage + (size_t)which * kPage + ts % kPage) * row_bytes)[c] = x;
+    }
+  }
+}
+
 // Shared-memory layout of one CTA (byte offsets from a 1024-aligned base).
 struct SmemLayout {
-  int stages, bars, misc, merge, prefix, sid, total;
+  int stages, bars, misc, merge, prefix, sid, step, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int ncw, int spw, int stage_bytes, int d, int S) {
+__host__ __device__ inline SmemLayout smem_layout(int ncw, int spw, int stage_bytes, int d, int S, bool step) {
   SmemLayout L;
   L.stages = 0;
   L.bars = ncw * spw * stage_bytes;
   L.misc = L.bars + 8 * ncw * spw;
-  L.merge = L.misc + 64;
+  L.merge = L.misc + 128;
   L.prefix = L.merge + ncw * kMaxGroup * (d + 2) * 4;
   L.sid = L.prefix + (S + 1) * 4;
-  L.total = L.sid + S * 4;
+  L.step = L.sid + S * 4;
+  L.total = L.step + (step ? 6 * S * 4 : 0);   // per-stream step decisions
   return L;
 }
 
@@ -432,22 +672,44 @@ __host__ __device__ inline SmemLayout smem_layout(int ncw, int spw, int stage_by
 // to finish it combines them (a few partials per stream). The next piece's
 // query is loaded before the merge, and the copies already in flight keep
 // HBM busy while the CTA merges.
-template <int D, int NCW, int NB, bool MMA, typename E>
-__global__ void __launch_bounds__(NCW * 32, 1)
+//
+// STEP: the launch also appends this step's token of every stream (the
+// decode step fused into one launch). The attention runs over the cache as
+// it was before the step: the row of the token that leaves at this step is
+// masked, and the new token enters every stream's final merge from its input
+// row. A ninth warp resolves each stream's slots (window ring, page pops in
+// stream order, the same rule as dms_append) and, once every CTA has read
+// the pre-step state (grid-wide counter), writes the append: bookkeeping and
+// the K/V rows. A row it overwrites is a masked one or lies past the
+// pre-step count, so no CTA ever attends a row being written.
+template <int D, int NCW, int NB, bool MMA, typename E, bool STEP>
+__global__ void __launch_bounds__((NCW + (STEP ? 1 : 0)) * 32, 1)
 attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
-  constexpr int kThreads = NCW * 32;
+  constexpr int kThreads = (NCW + (STEP ? 1 : 0)) * 32;   // consumers (+ the step warp)
+  constexpr int kMergeThreads = NCW * 32;                  // the consumer warps
   constexpr int kStage = 2 * kPage * D * (int)sizeof(E);   // one page: 16 K rows + 16 V rows
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int spw = a.spw;
-  const SmemLayout lay = smem_layout(NCW, spw, kStage, D, a.S);
+  const SmemLayout lay = smem_layout(NCW, spw, kStage, D, a.S, STEP);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
-  // misc: [0] abort, [1] ok, [2] last flag, [3 .. 3+NCW] scan scratch,
-  // [14] stream whose combine a split first piece left to the end of the range (-1: none)
+  // misc: [0] abort, [1] ok, [2] last flag, [3 .. 3+warps) scan scratch, [12] free-stack depth
+  // and [13] pages popped by this step (-1: pool exhausted), [14] stream whose combine a split
+  // first piece left to the end of the range (-1: none), [15] step decisions ready
   int* misc = reinterpret_cast<int*>(smem + lay.misc);
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(smem + lay.merge);
   int* prefix = reinterpret_cast<int*>(smem + lay.prefix);
   int* sid = reinterpret_cast<int*>(smem + lay.sid);
+  // STEP, per call stream: retained count and tokens seen before the step, the logical
+  // slot of the token leaving now (-1: none), the slot the new token takes (-1: not
+  // appended), flags (1 pops a page, 2 alpha, 4 bad seq id, 8 stream full, 16 pool
+  // exhausted) and the pop rank.
+  int* s_nold = reinterpret_cast<int*>(smem + lay.step);
+  int* s_pos = s_nold + a.S;
+  int* s_rslot = s_pos + a.S;
+  int* s_tslot = s_rslot + a.S;
+  int* s_flag = s_tslot + a.S;
+  int* s_rank = s_flag + a.S;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nst = a.n_seqs * a.hkv;
@@ -456,6 +718,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   if (tid == 0) {
     misc[0] = 0;
     misc[14] = -1;
+    misc[15] = 0;
     for (int s = 0; s < NCW * spw; ++s) mbar_init(smem_addr(&full[s]), 1);
     fence_mbar_init();
   }
@@ -468,17 +731,26 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   // in smem. The status word is read in the same round trip as the seq ids.
   {
     const int status = tid == 0 ? read_status(a.ctrl) : 0;
+    if (STEP && tid == 0) misc[12] = *reinterpret_cast<const volatile int32_t*>(&a.ctrl[kCtrlFree]);
     const int per = (nst + kThreads - 1) / kThreads;
     const int b0 = min(tid * per, nst), e0 = min(b0 + per, nst);
     int local = 0;
     for (int i = b0; i < e0; ++i) {
       const int seq = a.seq_ids[i / a.hkv];
+      const int al = STEP ? a.step.alpha[i] : 0;   // same round trip as the seq id
       int pages = 0, st = 0;
       if (seq < 0 || seq >= a.max_seqs) {
-        latch(a.ctrl, DMS_ERR_BAD_SEQ);
+        if constexpr (STEP) s_flag[i] = 4;   // latched once every CTA has read the status
+        else latch(a.ctrl, DMS_ERR_BAD_SEQ);
       } else {
         st = seq * a.hkv + i % a.hkv;
-        pages = (a.n[st] + kPage - 1) / kPage;
+        const int nn = a.n[st];
+        pages = (nn + kPage - 1) / kPage;
+        if constexpr (STEP) {
+          s_nold[i] = nn;
+          s_pos[i] = a.step.dv.pos[st];
+          s_flag[i] = al != 0 ? 2 : 0;
+        }
       }
       sid[i] = st;
       prefix[i + 1] = pages;
@@ -497,256 +769,316 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   }
   __syncthreads();
   grid_dependents_launch();   // the next kernel may queue up behind this one
-  if (!misc[1]) return;   // poisoned cache: do nothing (uniform over the CTA)
+  const bool healthy = misc[1] != 0;
+  if constexpr (!STEP) {
+    if (!healthy) return;   // poisoned cache: do nothing (uniform over the CTA)
+  }
   const long long P = prefix[nst];
   const int G = gridDim.x;
-
-  // Streams with nothing retained produce zeros.
-  for (int i = blockIdx.x; i < nst; i += G) {
-    if (prefix[i + 1] != prefix[i]) continue;
-    const int b = i / a.hkv, kvh = i % a.hkv;
-    for (int e = tid; e < a.g * D; e += kThreads) store_out(a, b, kvh * a.g + e / D, e % D, D, 0.f);
-  }
   const long long Geff = P < G ? P : G;
-  if (blockIdx.x >= Geff) return;   // uniform over the CTA
-  const int K0 = (int)(blockIdx.x * P / Geff), K1 = (int)((blockIdx.x + 1) * P / Geff);
+  if constexpr (!STEP) {
+    // Streams with nothing retained produce zeros.
+    for (int i = blockIdx.x; i < nst; i += G) {
+      if (prefix[i + 1] != prefix[i]) continue;
+      const int b = i / a.hkv, kvh = i % a.hkv;
+      for (int e = tid; e < a.g * D; e += kThreads) store_out(a, b, kvh * a.g + e / D, e % D, D, 0.f);
+    }
+    if (blockIdx.x >= Geff) return;   // uniform over the CTA
+  }
+  const bool has_range = healthy && blockIdx.x < Geff;
+  const int K0 = has_range ? (int)(blockIdx.x * P / Geff) : 0;
+  const int K1 = has_range ? (int)((blockIdx.x + 1) * P / Geff) : 0;
   const int ncta = K1 - K0;
+  int consumed = 0, issued = 0;
+  uint64_t* myfull = full + (warp < NCW ? warp : 0) * spw;
 
-  // ---- this warp's page pipeline: CTA pages c = warp + NCW * j, j = 0 .. njobs-1
-  const int njobs = ncta > warp ? (ncta - warp + NCW - 1) / NCW : 0;
-  uint64_t* myfull = full + warp * spw;
-  uint8_t* mystage = smem + lay.stages + (size_t)warp * spw * kStage;
-  auto lookup = [&](int j) -> int {   // physical page of the warp's j-th page
-    if (j >= njobs) return 0;
-    const int kk = K0 + warp + NCW * j;
-    const int i = stream_of(prefix, nst, kk);
-    int pg = __ldg(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i]));
-    if (pg < 0 || pg >= a.max_pages) {
-      latch(a.ctrl, DMS_ERR_INVALID);
-      pg = 0;
-    }
-    return pg;
-  };
-  int jb = 0;                                     // page ids of jobs [jb, jb+32) in pid_cur,
-  int pid_cur = lookup(lane), pid_nxt = lookup(32 + lane);   // [jb+32, jb+64) in pid_nxt
-  int issued = 0;
-  auto issue = [&](int j) {   // warp-uniform; j = issued
-    if (j - jb >= 32) {
-      pid_cur = pid_nxt;
-      jb += 32;
-      pid_nxt = lookup(jb + 32 + lane);
-    }
-    const int r = j - jb;
-    const int pg = __shfl_sync(0xffffffffu, r < 32 ? pid_cur : pid_nxt, r & 31);
-    if (lane == 0) {
-      const int s = j % spw;
-      const uint32_t bar = smem_addr(&myfull[s]);
-      const uint32_t dst = smem_addr(mystage + (size_t)s * kStage);
-      mbar_arrive_expect_tx(bar, kStage);
-      if constexpr (MMA) {
+  if (STEP && warp == NCW) {
+    step_warp<D, E>(a, nst, prefix, sid, s_nold, s_pos, s_rslot, s_tslot, s_flag, s_rank, misc, healthy,
+                    abort_flag);
+  } else if (STEP || has_range) {
+    // ---- this warp's page pipeline: CTA pages c = warp + NCW * j, j = 0 .. njobs-1
+    const int njobs = has_range && ncta > warp ? (ncta - warp + NCW - 1) / NCW : 0;
+    uint8_t* mystage = smem + lay.stages + (size_t)warp * spw * kStage;
+    auto lookup = [&](int j) -> int {   // physical page of the warp's j-th page
+      if (j >= njobs) return 0;
+      const int kk = K0 + warp + NCW * j;
+      const int i = stream_of(prefix, nst, kk);
+      int pg = __ldg(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i]));
+      if (pg < 0 || pg >= a.max_pages) {
+        latch(a.ctrl, DMS_ERR_INVALID);
+        pg = 0;
+      }
+      return pg;
+    };
+    using State = typename std::conditional<MMA, MmaState<D>, SimtState<D>>::type;
+    using Query = typename std::conditional<MMA, MmaQuery<D>, SimtQuery<D>>::type;
+    State S;
+    Query qcur;
+    auto fetch_query = [&](int stream) {
+      if constexpr (MMA) mma_fetch_q<D>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
+      else simt_fetch_q<D, E>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
+    };
+    auto start_piece = [&]() {   // take the fetched query, clear the softmax state
+      if constexpr (MMA) mma_start<D>(S, qcur);
+      else simt_start<D>(S, qcur);
+    };
+    auto load_query = [&](int stream) {
+      fetch_query(stream);
+      start_piece();
+    };
+    // The first piece's query is requested in the same round trip as the page
+    // ids, before the copies fill the memory queues.
+    int i = has_range ? stream_of(prefix, nst, K0) : 0;
+    if (has_range) fetch_query(i);
+    // STEP: the window-ring entry of every call stream (the token at s - w),
+    // requested before the page ids so that both land before the first copies
+    // are issued: a load queued behind the grid's first burst of page copies
+    // waits microseconds.
+    constexpr int kRingPer = (kStepMaxStreams + kMergeThreads - 1) / kMergeThreads;
+    int ring_v[STEP ? kRingPer : 1];
+    if constexpr (STEP) {
 #pragma unroll
-        for (int box = 0; box < D / 64; ++box) tma_load_3d(dst + box * 4096, &tmap, bar, box * 64, 0, pg);
-      } else {
-        bulk_load(dst, a.kv + (size_t)pg * kStage, kStage, bar);
+      for (int q = 0; q < kRingPer; ++q) {
+        const int il = tid + q * kMergeThreads;
+        ring_v[q] = (il < nst && !(s_flag[il] & 4))
+                        ? ld_early(a.step.dv.ring + (size_t)sid[il] * a.step.dv.w + (s_pos[il] % a.step.dv.w))
+                        : 0;
       }
     }
-    issued = j + 1;
-  };
-  for (int j = 0; j < spw && j < njobs; ++j) issue(j);
-
-  using State = typename std::conditional<MMA, MmaState<D>, SimtState<D>>::type;
-  using Query = typename std::conditional<MMA, MmaQuery<D>, SimtQuery<D>>::type;
-  State S;
-  Query qcur;
-  auto load_query = [&](int stream) {   // the piece's query; clears the softmax state
-    if constexpr (MMA) {
-      mma_fetch_q<D>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
-      mma_start<D>(S, qcur);
-    } else {
-      simt_fetch_q<D, E>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
-      simt_start<D>(S, qcur);
-    }
-  };
-  const MmaOffsets<D> off(lane);
-  int consumed = 0;
-  int k = K0;
-  int i = stream_of(prefix, nst, k);
-  load_query(i);
-  int nn = __ldg(a.n + sid[i]);
-  while (k < K1) {
-    const int pstart = prefix[i], pend = prefix[i + 1];
-    const int pe = min(pend, K1);
-    const int b = i / a.hkv, kvh = i % a.hkv;
-    const bool whole = (k == pstart) && (pe == pend);
-
-    const int rel = k - K0;
-    for (int c = rel + ((warp - rel) % NCW + NCW) % NCW; c < pe - K0;) {
-      const int j = (c - warp) / NCW;
-      const int nb = (NB == 2 && c + NCW < pe - K0) ? 2 : 1;   // pages in this batch (same stream)
-      bool ok = mbar_wait_bounded(smem_addr(&myfull[j % spw]), (j / spw) & 1, abort_flag, a.ctrl);
-      if (nb == 2) ok &= mbar_wait_bounded(smem_addr(&myfull[(j + 1) % spw]), ((j + 1) / spw) & 1, abort_flag, a.ctrl);
-      if (ok) {
-        const int p = K0 + c - pstart;   // page index within the stream
-        const int valid0 = (K0 + c == pend - 1) ? nn - kPage * p : kPage;
-        const uint8_t* st0 = mystage + (size_t)(j % spw) * kStage;
+    int jb = 0;                                     // page ids of jobs [jb, jb+32) in pid_cur,
+    int pid_cur = lookup(lane), pid_nxt = lookup(32 + lane);   // [jb+32, jb+64) in pid_nxt
+    auto issue = [&](int j) {   // warp-uniform; j = issued
+      if (j - jb >= 32) {
+        pid_cur = pid_nxt;
+        jb += 32;
+        pid_nxt = lookup(jb + 32 + lane);
+      }
+      const int r = j - jb;
+      const int pg = __shfl_sync(0xffffffffu, r < 32 ? pid_cur : pid_nxt, r & 31);
+      if (lane == 0) {
+        const int s = j % spw;
+        const uint32_t bar = smem_addr(&myfull[s]);
+        const uint32_t dst = smem_addr(mystage + (size_t)s * kStage);
+        mbar_arrive_expect_tx(bar, kStage);
         if constexpr (MMA) {
-          if (nb == 2) {
-            const int valid1 = (K0 + c + NCW == pend - 1) ? nn - kPage * (p + NCW) : kPage;
-            const uint32_t stg[2] = {smem_addr(st0), smem_addr(mystage + (size_t)((j + 1) % spw) * kStage)};
-            const int val[2] = {valid0, valid1};
-            mma_pages<D, 2>(S, stg, val, a.sl2e, lane, off);
-          } else {
-            const uint32_t stg[1] = {smem_addr(st0)};
-            const int val[1] = {valid0};
-            mma_pages<D, 1>(S, stg, val, a.sl2e, lane, off);
-          }
+#pragma unroll
+          for (int box = 0; box < D / 64; ++box) tma_load_3d(dst + box * 4096, &tmap, bar, box * 64, 0, pg);
         } else {
-          simt_page<D, E>(S, reinterpret_cast<const E*>(st0), valid0, a.g, lane);
+          bulk_load(dst, a.kv + (size_t)pg * kStage, kStage, bar);
         }
       }
-      consumed = j + nb;
-      __syncwarp();
-      const bool stop = __any_sync(0xffffffffu, *abort_flag != 0);
-      for (int q = 0; q < nb; ++q)
-        if (j + q + spw < njobs && !stop) issue(j + q + spw);
-      c += nb * NCW;
-    }
-
-    // ---- end of the piece: merge the warps' states in shared memory
-    if constexpr (MMA) mma_to_slot<D>(S, &slots[warp], lane);
-    else simt_to_slot<D>(S, &slots[warp], lane);
-    // start loading the next piece's query while the CTA merges
-    const int inext = pe < K1 ? stream_of(prefix, nst, pe) : i;
-    if (pe < K1) load_query(inext);
-    const int nn_next = pe < K1 ? __ldg(a.n + sid[inext]) : 0;
-    __syncthreads();
-
-    // Merge: thread t owns query head h = t / (D/4) and dims [4 d4, 4 d4 + 4);
-    // the CTA's result for its items stays in registers for the combine.
-    constexpr int kItems = kMaxGroup * D / 4;
-    constexpr int kIters = (kItems + kThreads - 1) / kThreads;
-    const int items = a.g * (D / 4);
-    float4 myO[kIters];
-    float myM[kIters], myL[kIters];
-    Partial<D>* part = reinterpret_cast<Partial<D>*>(a.part) + (blockIdx.x + i);
+      issued = j + 1;
+    };
+    for (int j = 0; j < spw && j < njobs; ++j) issue(j);
+    if constexpr (STEP) {
+      // The logical slot of the token leaving at this step (-1: none), for the
+      // consumers' masks and the step warp's decisions.
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const int t = tid + it * kThreads;
-      if (t >= items) break;
-      const int h = t / (D / 4), d4 = t % (D / 4);
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) M = fmaxf(M, slots[w].m[h]);
-      float L = 0.f;
-      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const float sc = ex2(slots[w].m[h] - M);   // 0 for a warp that saw nothing (m = -inf)
-        const float4 o = *reinterpret_cast<const float4*>(&slots[w].O[h][4 * d4]);
-        L = fmaf(slots[w].l[h], sc, L);
-        O.x = fmaf(o.x, sc, O.x);
-        O.y = fmaf(o.y, sc, O.y);
-        O.z = fmaf(o.z, sc, O.z);
-        O.w = fmaf(o.w, sc, O.w);
+      for (int q = 0; q < kRingPer; ++q) {
+        const int il = tid + q * kMergeThreads;
+        if (il < nst && !(s_flag[il] & 4))
+          s_rslot[il] = (s_pos[il] >= a.step.dv.w && (ring_v[q] & 1)) ? (ring_v[q] >> 1) : -1;
+        else if (il < nst)
+          s_rslot[il] = -1;
       }
-      if (whole) {
-        store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, 1.f / L);
-      } else {
-        __stcg(reinterpret_cast<float4*>(&part->O[h][4 * d4]), O);
-        if (d4 == 0) {
-          __stcg(&part->m[h], M);
-          __stcg(&part->l[h], L);
+      named_barrier_arrive(2, kThreads);   // hand them to the step warp (which syncs on barrier 2)
+    }
+    if (has_range) {
+
+
+      auto retained_of = [&](int stream) -> int {   // retained count the attention runs over
+        if constexpr (STEP) return s_nold[stream];
+        else return __ldg(a.n + sid[stream]);
+      };
+      const MmaOffsets<D> off(lane);
+      int k = K0;
+      start_piece();
+      int nn = retained_of(i);
+      bool decisions = false;   // STEP: the step warp's decisions have been seen
+      auto await_decisions = [&]() {
+        if (STEP && !decisions) {
+          if (lane == 0) wait_flag_ge(misc + 15, 1, abort_flag, a.ctrl);
+          __syncwarp();
+          __threadfence_block();
+          decisions = true;
         }
-        myO[it] = O;
-        myM[it] = M;
-        myL[it] = L;
-      }
-    }
-    __syncthreads();   // the slots are read and the partial (if any) is complete
-    if (!whole) {
-      // Publish the partial: the CTA's stores, ordered by the barrier, are
-      // released by thread 0's device-scope add; the adder that completes the
-      // count acquires every other piece and combines.
-      const int first = range_of(pstart, P, Geff), last = range_of(pend - 1, P, Geff);
-      if (pe < K1) {
-        // A split piece inside the range is its first piece. Thread 0
-        // publishes it while the CTA goes on; a combine it finds due is done
-        // by the whole CTA at the end of the range.
-        if (tid == 0 && atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first) misc[14] = i;
-      } else {
-        if (tid == 0) misc[2] = (atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first);
-        __syncthreads();
-        if (misc[2]) {
-          const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
-          const int me = blockIdx.x;
-#pragma unroll
-          for (int it = 0; it < kIters; ++it) {
-            const int t = tid + it * kThreads;
-            if (t >= items) break;
-            const int h = t / (D / 4), d4 = t % (D / 4);
-            float M = myM[it], L = myL[it];
-            float4 O = myO[it];
-            for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
-              float mc[4], lc[4];
-              float4 oc[4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int c = c0 + u;
-                const bool use = c <= last && c != me;
-                mc[u] = use ? __ldcg(&base[c].m[h]) : -INFINITY;
-                lc[u] = use ? __ldcg(&base[c].l[h]) : 0.f;
-                oc[u] = use ? __ldcg(reinterpret_cast<const float4*>(&base[c].O[h][4 * d4]))
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      };
+      while (k < K1) {
+        const int pstart = prefix[i], pend = prefix[i + 1];
+        const int pe = min(pend, K1);
+        const int b = i / a.hkv, kvh = i % a.hkv;
+        const bool whole = (k == pstart) && (pe == pend);
+        const int rslot = STEP ? s_rslot[i] : -1;   // row of the token leaving at this step
+        auto rows_of = [&](int p) -> uint32_t {      // rows to attend in page p of the stream
+          const int valid = (pstart + p == pend - 1) ? nn - kPage * p : kPage;
+          uint32_t r = valid >= kPage ? 0xffffu : ((1u << valid) - 1u);
+          if (rslot >= 0 && (rslot >> 4) == p) r &= ~(1u << (rslot & 15));
+          return r;
+        };
+
+        const int rel = k - K0;
+        for (int c = rel + ((warp - rel) % NCW + NCW) % NCW; c < pe - K0;) {
+          const int j = (c - warp) / NCW;
+          const int nb = (NB == 2 && c + NCW < pe - K0) ? 2 : 1;   // pages in this batch (same stream)
+          bool ok = mbar_wait_bounded(smem_addr(&myfull[j % spw]), (j / spw) & 1, abort_flag, a.ctrl);
+          if (nb == 2) ok &= mbar_wait_bounded(smem_addr(&myfull[(j + 1) % spw]), ((j + 1) / spw) & 1, abort_flag, a.ctrl);
+          if (ok) {
+            const int p = K0 + c - pstart;   // page index within the stream
+            const uint8_t* st0 = mystage + (size_t)(j % spw) * kStage;
+            if constexpr (MMA) {
+              if (nb == 2) {
+                const uint32_t stg[2] = {smem_addr(st0), smem_addr(mystage + (size_t)((j + 1) % spw) * kStage)};
+                const uint32_t rw[2] = {rows_of(p), rows_of(p + NCW)};
+                mma_pages<D, 2>(S, stg, rw, a.sl2e, lane, off);
+              } else {
+                const uint32_t stg[1] = {smem_addr(st0)};
+                const uint32_t rw[1] = {rows_of(p)};
+                mma_pages<D, 1>(S, stg, rw, a.sl2e, lane, off);
               }
-#pragma unroll
-              for (int u = 0; u < 4; ++u) merge_into(M, L, O, mc[u], lc[u], oc[u]);
+            } else {
+              simt_page<D, E>(S, reinterpret_cast<const E*>(st0), rows_of(p), a.g, lane);
             }
-            store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, 1.f / L);
           }
-          if (tid == 0) a.cnt[i] = 0;   // ready for the next launch (stream order)
+          consumed = j + nb;
+          __syncwarp();
+          const bool stop = __any_sync(0xffffffffu, *abort_flag != 0);
+          for (int q = 0; q < nb; ++q)
+            if (j + q + spw < njobs && !stop) issue(j + q + spw);
+          c += nb * NCW;
         }
+
+        // ---- end of the piece: merge the warps' states in shared memory
+        if constexpr (MMA) mma_to_slot<D>(S, &slots[warp], lane);
+        else simt_to_slot<D>(S, &slots[warp], lane);
+        // start loading the next piece's query while the CTA merges
+        const int inext = pe < K1 ? stream_of(prefix, nst, pe) : i;
+        if (pe < K1) load_query(inext);
+        const int nn_next = pe < K1 ? retained_of(inext) : 0;
+        named_barrier(1, kMergeThreads);
+
+        // Merge: thread t owns query head h = t / (D/4) and dims [4 d4, 4 d4 + 4);
+        // the CTA's result for its items stays in registers for the combine.
+        constexpr int kItems = kMaxGroup * D / 4;
+        constexpr int kIters = (kItems + kMergeThreads - 1) / kMergeThreads;
+        const int items = a.g * (D / 4);
+        if (STEP) await_decisions();
+        const bool add_new = STEP && s_tslot[i] >= 0;   // the stream's new token (appended by this step)
+        float4 myO[kIters];
+        float myM[kIters], myL[kIters];
+        Partial<D>* part = reinterpret_cast<Partial<D>*>(a.part) + (blockIdx.x + i);
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+          const int t = tid + it * kMergeThreads;
+          const bool live = t < items;
+          if (!__any_sync(0xffffffffu, live)) break;   // warp-uniform
+          const int h = (live ? t : 0) / (D / 4), d4 = (live ? t : 0) % (D / 4);
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < NCW; ++w) M = fmaxf(M, slots[w].m[h]);
+          float L = 0.f;
+          float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int w = 0; w < NCW; ++w) {
+            // 0 for a warp that saw nothing (m = -inf); all 0 if no warp saw a token
+            const float sc = M == -INFINITY ? 0.f : ex2(slots[w].m[h] - M);
+            const float4 o = *reinterpret_cast<const float4*>(&slots[w].O[h][4 * d4]);
+            L = fmaf(slots[w].l[h], sc, L);
+            O.x = fmaf(o.x, sc, O.x);
+            O.y = fmaf(o.y, sc, O.y);
+            O.z = fmaf(o.z, sc, O.z);
+            O.w = fmaf(o.w, sc, O.w);
+          }
+          if (whole) {
+            if constexpr (STEP) add_new_token<D, E>(a, i, h, d4, add_new, M, L, O);   // warp-collective
+            if (live) store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, L > 0.f ? 1.f / L : 0.f);
+          } else if (live) {
+            __stcg(reinterpret_cast<float4*>(&part->O[h][4 * d4]), O);
+            if (d4 == 0) {
+              __stcg(&part->m[h], M);
+              __stcg(&part->l[h], L);
+            }
+            myO[it] = O;
+            myM[it] = M;
+            myL[it] = L;
+          }
+        }
+        named_barrier(1, kMergeThreads);   // the slots are read and the partial (if any) is complete
+        if (!whole) {
+          // Publish the partial: the CTA's stores, ordered by the barrier, are
+          // released by thread 0's device-scope add; the adder that completes the
+          // count acquires every other piece and combines.
+          const int first = range_of(pstart, P, Geff), last = range_of(pend - 1, P, Geff);
+          if (pe < K1) {
+            // A split piece inside the range is its first piece. Thread 0
+            // publishes it while the CTA goes on; a combine it finds due is done
+            // by the whole CTA at the end of the range.
+            if (tid == 0 && atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first) misc[14] = i;
+          } else {
+            if (tid == 0) misc[2] = (atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first);
+            named_barrier(1, kMergeThreads);
+            if (misc[2]) {
+              const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
+              const int me = blockIdx.x;
+#pragma unroll
+              for (int it = 0; it < kIters; ++it) {
+                const int t = tid + it * kMergeThreads;
+                const bool live = t < items;
+                if (!__any_sync(0xffffffffu, live)) break;   // warp-uniform
+                const int h = (live ? t : 0) / (D / 4), d4 = (live ? t : 0) % (D / 4);
+                float M = live ? myM[it] : 0.f, L = live ? myL[it] : 1.f;
+                float4 O = live ? myO[it] : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
+                  float mc[4], lc[4];
+                  float4 oc[4];
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + u;
+                    const bool use = c <= last && c != me;
+                    mc[u] = use ? __ldcg(&base[c].m[h]) : -INFINITY;
+                    lc[u] = use ? __ldcg(&base[c].l[h]) : 0.f;
+                    oc[u] = use ? __ldcg(reinterpret_cast<const float4*>(&base[c].O[h][4 * d4]))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                  }
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) merge_into(M, L, O, mc[u], lc[u], oc[u]);
+                }
+                if constexpr (STEP) add_new_token<D, E>(a, i, h, d4, add_new, M, L, O);   // warp-collective
+                if (live) store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, L > 0.f ? 1.f / L : 0.f);
+              }
+              if (tid == 0) a.cnt[i] = 0;   // ready for the next launch (stream order)
+            }
+          }
+        }
+        k = pe;
+        i = inext;
+        nn = nn_next;
       }
     }
-    k = pe;
-    i = inext;
-    nn = nn_next;
   }
 
   // ---- a split first piece that completed its stream: combine all its pieces
   __syncthreads();
-  if (misc[14] >= 0) {
+  if (tid < kMergeThreads && misc[14] >= 0) {
     const int i = misc[14];
     const int first = range_of(prefix[i], P, Geff), last = range_of(prefix[i + 1] - 1, P, Geff);
-    const int b = i / a.hkv, kvh = i % a.hkv;
-    const int items = a.g * (D / 4);
-    const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
-    for (int t = tid; t < items; t += kThreads) {
-      const int h = t / (D / 4), d4 = t % (D / 4);
-      float M = -INFINITY, L = 0.f;
-      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
-        float mc[4], lc[4];
-        float4 oc[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int c = c0 + u;
-          mc[u] = c <= last ? __ldcg(&base[c].m[h]) : -INFINITY;
-          lc[u] = c <= last ? __ldcg(&base[c].l[h]) : 0.f;
-          oc[u] = c <= last ? __ldcg(reinterpret_cast<const float4*>(&base[c].O[h][4 * d4]))
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (c0 + u <= last) merge_into(M, L, O, mc[u], lc[u], oc[u]);
-      }
-      store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, 1.f / L);
-    }
+    combine_stream<D, E, STEP>(a, i, first, last, tid, kMergeThreads, STEP && s_tslot[i] >= 0);
     if (tid == 0) a.cnt[i] = 0;   // ready for the next launch (stream order)
   }
 
   // Drain: copies issued but not consumed (only after an abort) must land before exit.
-  if (lane == 0)
+  if (warp < NCW && lane == 0)
     for (int j = consumed; j < issued; ++j) mbar_wait_timed(smem_addr(&myfull[j % spw]), (j / spw) & 1, a.ctrl);
+
+  if constexpr (STEP) {
+    // The last CTA out resets the step's grid counters for the next launch.
+    __syncthreads();
+    if (tid == 0) {
+      if (atomic_add_acq_rel_gpu(&a.ctrl[kCtrlExited], 1) == (int)gridDim.x - 1) {
+        a.ctrl[kCtrlPlanned] = 0;
+        a.ctrl[kCtrlExited] = 0;
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -754,20 +1086,21 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
 
 using KernelFn = void (*)(const AttnArgs, const __grid_constant__ CUtensorMap);
 
-template <int D, int NCW, int NB, bool MMA, typename E>
-KernelFn kernel_ptr() { return attn_kernel<D, NCW, NB, MMA, E>; }
+template <int D, int NCW, int NB, bool MMA, typename E, bool STEP>
+KernelFn kernel_ptr() { return attn_kernel<D, NCW, NB, MMA, E, STEP>; }
 
-template <int NB, bool MMA, typename E>
+template <int NB, bool MMA, typename E, bool STEP>
 KernelFn pick_ncw(int d, int ncw) {
-  if (d == 64) return ncw == 4 ? kernel_ptr<64, 4, NB, MMA, E>() : kernel_ptr<64, 8, NB, MMA, E>();
-  return ncw == 4 ? kernel_ptr<128, 4, NB, MMA, E>() : kernel_ptr<128, 8, NB, MMA, E>();
+  if (d == 64) return ncw == 4 ? kernel_ptr<64, 4, NB, MMA, E, STEP>() : kernel_ptr<64, 8, NB, MMA, E, STEP>();
+  return ncw == 4 ? kernel_ptr<128, 4, NB, MMA, E, STEP>() : kernel_ptr<128, 8, NB, MMA, E, STEP>();
 }
 
+template <bool STEP>
 KernelFn pick_kernel(int d, int dtype, int kernel, int ncw, int nb) {
   if (kernel == DMS_ATTN_MMA)
-    return nb == 2 ? pick_ncw<2, true, uint16_t>(d, ncw) : pick_ncw<1, true, uint16_t>(d, ncw);
-  if (dtype == DMS_BF16) return pick_ncw<1, false, uint16_t>(d, ncw);
-  return pick_ncw<1, false, float>(d, ncw);
+    return nb == 2 ? pick_ncw<2, true, uint16_t, STEP>(d, ncw) : pick_ncw<1, true, uint16_t, STEP>(d, ncw);
+  if (dtype == DMS_BF16) return pick_ncw<1, false, uint16_t, STEP>(d, ncw);
+  return pick_ncw<1, false, float, STEP>(d, ncw);
 }
 
 int env_int(const char* name, int dflt) {
@@ -779,9 +1112,8 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-}  // namespace
 
-cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan) {
+cudaError_t prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, bool step, AttnPlan* plan) {
   int kernel = kernel_choice;
   if (kernel == DMS_ATTN_AUTO) kernel = (dtype == DMS_BF16) ? DMS_ATTN_MMA : DMS_ATTN_SIMT;
   if (kernel == DMS_ATTN_MMA && dtype != DMS_BF16) return cudaErrorInvalidValue;
@@ -798,19 +1130,19 @@ cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int n
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&per_block_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
   const int budget = std::min(per_block_smem, per_sm_smem / ctas - 1024) - 1024;   // minus alignment slack
-  const int fixed = smem_layout(ncw, 0, stage_bytes, dv.d, dv.S).total;
+  const int fixed = smem_layout(ncw, 0, stage_bytes, dv.d, dv.S, step).total;
   int spw = std::min(8, (budget - fixed) / (ncw * stage_bytes));
   const int want = env_int("DMS_ATTN_STAGES", 0);
   if (want > 0) spw = std::min(spw, want);
   if (spw < nb) return cudaErrorInvalidConfiguration;
 
-  KernelFn fn = pick_kernel(dv.d, dtype, kernel, ncw, nb);
+  KernelFn fn = step ? pick_kernel<true>(dv.d, dtype, kernel, ncw, nb) : pick_kernel<false>(dv.d, dtype, kernel, ncw, nb);
   plan->kernel = kernel;
   plan->ncw = ncw;
   plan->spw = spw;
   plan->fn = reinterpret_cast<void*>(fn);
-  plan->threads = ncw * 32;
-  plan->smem = 1024 + (size_t)smem_layout(ncw, spw, stage_bytes, dv.d, dv.S).total;
+  plan->threads = (ncw + (step ? 1 : 0)) * 32;
+  plan->smem = 1024 + (size_t)smem_layout(ncw, spw, stage_bytes, dv.d, dv.S, step).total;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan->smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
@@ -841,11 +1173,23 @@ cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int n
   return cudaSuccess;
 }
 
-cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,
-                             const int32_t* seq_ids, const void* Q, int hq, float scale, void* out,
-                             int out_f32) {
-  if (n_seqs == 0) return cudaSuccess;
+
+}  // namespace
+
+cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan) {
+  return prepare(dv, dtype, kernel_choice, num_sms, false, plan);
+}
+
+cudaError_t step_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan) {
+  return prepare(dv, dtype, kernel_choice, num_sms, true, plan);
+}
+
+namespace {
+
+AttnArgs attn_args(const Dev& dv, const AttnPlan& plan, int n_seqs, const int32_t* seq_ids, const void* Q,
+                   int hq, float scale, void* out, int out_f32) {
   AttnArgs a;
+  memset(&a, 0, sizeof(a));
   a.seq_ids = seq_ids;
   a.Q = (const uint8_t*)Q;
   a.out = (uint8_t*)out;
@@ -866,6 +1210,29 @@ cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t s
   a.sl2e = scale * kLog2e;
   a.spw = plan.spw;
   a.S = dv.S;
+  return a;
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,
+                             const int32_t* seq_ids, const void* Q, int hq, float scale, void* out,
+                             int out_f32) {
+  if (n_seqs == 0) return cudaSuccess;
+  const AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32);
+  return launch_dependent(reinterpret_cast<KernelFn>(plan.fn), dim3(plan.grid), dim3(plan.threads), plan.smem, st,
+                          a, plan.tmap);
+}
+
+cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
+                        const void* K, const void* V, const uint8_t* alpha, const void* Q, int hq, float scale,
+                        void* out, int out_f32) {
+  if (n_seqs == 0) return cudaSuccess;
+  AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32);
+  a.step.K = (const uint8_t*)K;
+  a.step.V = (const uint8_t*)V;
+  a.step.alpha = alpha;
+  a.step.dv = dv;
   return launch_dependent(reinterpret_cast<KernelFn>(plan.fn), dim3(plan.grid), dim3(plan.threads), plan.smem, st,
                           a, plan.tmap);
 }

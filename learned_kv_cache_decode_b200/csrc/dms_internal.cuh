@@ -20,7 +20,8 @@ constexpr int kMaxKvHeads = 256;
 enum : int {
   kCtrlStatus = 0,   // latched dms_status, 0 = healthy
   kCtrlFree = 1,     // free-stack depth
-  kCtrlArrive = 2,   // arrival counter of the decode-append kernel
+  kCtrlPlanned = 2,  // CTAs of a fused decode step done reading the pre-step state
+  kCtrlExited = 3,   // CTAs of a fused decode step that finished
   kCtrlWords = 8
 };
 
@@ -136,6 +137,24 @@ __device__ __forceinline__ void mbar_wait_timed(uint32_t bar, uint32_t parity, i
   }
 }
 
+// Spin (one thread) until *flag >= target, bounded by ~2^31 SM cycles; on
+// timeout latch DMS_ERR_TIMEOUT and raise the CTA's abort flag. Gives up at
+// once when the abort flag is already up. sleep_ns > 0 sleeps between polls.
+__device__ __forceinline__ void wait_flag_ge(volatile int* flag, int target, volatile int* abort_flag,
+                                             int32_t* ctrl, int sleep_ns = 0) {
+  if (*flag >= target) return;
+  const long long t0 = clock64();
+  while (*flag < target) {
+    if (sleep_ns) __nanosleep(sleep_ns);   // leave the issue slots to the warps doing work
+    if (*abort_flag) return;
+    if (clock64() - t0 > (1ll << 31)) {
+      latch(ctrl, DMS_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return;
+    }
+  }
+}
+
 // TMA tiled load of a 3-D box into shared memory, completing on an mbarrier.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int x, int y, int z) {
@@ -207,6 +226,15 @@ __device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
   return old;
 }
 
+// A global load that stays where it is written, ahead of the asm volatile
+// statements that follow it (the TMA copies), instead of being sunk next to
+// its first use behind them.
+__device__ __forceinline__ int ld_early(const int32_t* p) {
+  int v;
+  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Programmatic dependent launch. A kernel launched with launch_dependent()
 // may start while the previous kernel of its stream is still running; it
 // must call grid_dependency_wait() before it touches memory that earlier
@@ -230,6 +258,24 @@ inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
+
+// Arrive at a named barrier without waiting (the producer side of a
+// producer/consumer hand-off; the consumers bar.sync on it). Stores before the
+// arrival are visible to the threads that sync on the barrier.
+__device__ __forceinline__ void named_barrier_arrive(int id, int threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Device-scope add with release semantics (no return value): the caller's
+// earlier memory operations, and those of its CTA ordered before it by a
+// barrier, happen before any acquire that observes the add.
+__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Acquire-release fence at device scope (weaker and cheaper than the
+// sequentially consistent fence of __threadfence).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -264,6 +310,13 @@ struct AttnPlan {
 };
 
 cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan);
+// The fused decode step (append + attention in one launch); see dms_decode_step.
+cudaError_t step_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan);
+cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
+                        const void* K, const void* V, const uint8_t* alpha, const void* Q, int hq, float scale,
+                        void* out, int out_f32);
+constexpr int kStepMaxStreams = 1024;   // caches with more streams run the step as two launches
+
 cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,
                              const int32_t* seq_ids, const void* Q, int hq, float scale, void* out,
                              int out_f32);

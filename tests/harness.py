@@ -104,10 +104,22 @@ class Run:
         Q = W.query(self.wl, step)[list(seqs)]
         return K, V, A, Q
 
-    def decode_step(self, step: int, seqs=None, out_dtype=None):
+    def decode_step(self, step: int, seqs=None, out_dtype=None, fused: bool = False):
+        """Append one token per sequence and attend: two launches (dms_append then
+        dms_decode_attention) or, with `fused`, one dms_decode_step."""
         seqs = list(range(self.wl.batch)) if seqs is None else list(seqs)
         K, V, A, Q = self.decode_inputs(step, seqs)
         ids = torch.tensor(seqs, dtype=torch.int32, device="cuda")
+        if fused:
+            out = self.cache.decode_step(ids, to_device(K, self.wl), to_device(V, self.wl),
+                                         torch.from_numpy(A).cuda(), to_device(Q, self.wl), scale=self.scale,
+                                         out_dtype=out_dtype)
+            if self.sim is not None:
+                rc, _ = self.sim.append(seqs, [1] * len(seqs), A)
+                assert rc == 0, rc
+            for b in seqs:
+                self.seen[b] += 1
+            return out, Q
         self.cache.append(ids, to_device(K, self.wl), to_device(V, self.wl), torch.from_numpy(A).cuda())
         if self.sim is not None:
             rc, _ = self.sim.append(seqs, [1] * len(seqs), A)

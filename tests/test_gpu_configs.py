@@ -16,7 +16,7 @@ from harness import Run, compare
 pytestmark = pytest.mark.gpu
 
 
-def _run_config(name, check_steps, check_seqs, steps=None, chunk=4096, metadata_every=None):
+def _run_config(name, check_steps, check_seqs, steps=None, chunk=4096, metadata_every=None, fused=False):
     wl = W.WORKLOADS[name]
     run = Run(wl, steps=steps)
     try:
@@ -24,7 +24,7 @@ def _run_config(name, check_steps, check_seqs, steps=None, chunk=4096, metadata_
         run.check_metadata()
         n = run.steps
         for step in range(n):
-            out, Q = run.decode_step(step)
+            out, Q = run.decode_step(step, fused=fused)
             if step in check_steps:
                 torch.cuda.synchronize()
                 for b in check_seqs:
@@ -95,3 +95,13 @@ def test_longrun_2k_30k():
         assert run.cache.status() == _native.DMS_OK
     finally:
         run.close()
+
+
+def test_qwen_r1_7b_32k_fused_step():
+    """The same workload through dms_decode_step (append and attention in one launch)."""
+    _run_config("qwen-r1-7b-32k", check_steps={0, 255}, check_seqs=[0, 7, 15], metadata_every=128, fused=True)
+
+
+def test_qwen_r1_32b_chains_fused_step():
+    _run_config("qwen-r1-32b-chains", check_steps={0, 255}, check_seqs=[0, 21, 63], metadata_every=128,
+                fused=True)

@@ -210,3 +210,97 @@ def test_host_argument_checks():
         args.update(bad)
         with pytest.raises(_native.DmsError):
             DmsCache(**args)
+
+
+# ---------------------------------------------------------------------------
+# dms_decode_step: append and attention fused into one launch
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c.name for c in CASES])
+def test_small_cases_fused_step(case):
+    """The fused step against the oracle: metadata bit for bit, outputs within tolerance."""
+    for kern in kernels_for(case):
+        run = Run(case, attn_kernel=kern)
+        try:
+            run.prefill(chunk=97)
+            run.check_metadata()
+            for step in range(case.decode_steps):
+                out, Q = run.decode_step(step, fused=True)
+                torch.cuda.synchronize()
+                for b in range(case.batch):
+                    ref = run.oracle_out(b, Q[b])
+                    tol = dict(max_abs=1e-4, mean_abs=1e-5) if case.dtype == "f32" else {}
+                    compare(out[b], ref, **tol)
+                run.check_metadata()
+            assert run.cache.status() == _native.DMS_OK
+        finally:
+            run.close()
+
+
+def test_fused_step_equals_two_launches():
+    """Same inputs through dms_decode_step and through dms_append + dms_decode_attention:
+    identical bookkeeping and pool rows, outputs equal to fp32 rounding order."""
+    case = wl("fused-vs-two", 4, 28, 4, 128, "bf16", 24, (1, 800), 40, 0.7, 31)
+    a, b = Run(case), Run(case, check_sim=False)
+    try:
+        a.prefill(chunk=200)
+        b.prefill(chunk=200)
+        for step in range(case.decode_steps):
+            oa, _ = a.decode_step(step)
+            ob, _ = b.decode_step(step, fused=True)
+            torch.cuda.synchronize()
+            diff = (oa.float() - ob.float()).abs()
+            assert float(diff.max()) <= 1e-2 and float(diff.mean()) <= 1e-3
+        sa, sb = a.cache.snapshot(), b.cache.snapshot()
+        for k in ("n", "pos", "n_pages", "page_table", "free_list"):
+            np.testing.assert_array_equal(sa[k], sb[k], err_msg=k)
+        assert sa["free_count"] == sb["free_count"]
+        for st in range(case.streams):
+            n = int(sa["n"][st])
+            if n:
+                ka, va = a.cache.gather_kv(st // case.num_kv_heads, st % case.num_kv_heads, n)
+                kb, vb = b.cache.gather_kv(st // case.num_kv_heads, st % case.num_kv_heads, n)
+                assert torch.equal(ka, kb) and torch.equal(va, vb)
+        assert a.cache.status() == _native.DMS_OK and b.cache.status() == _native.DMS_OK
+    finally:
+        a.close()
+        b.close()
+
+
+def test_fused_step_pool_exhaustion_matches_two_launches():
+    """A pool too small for this step's page pops: both paths latch POOL_EXHAUSTED and
+    leave the same bookkeeping (streams that needed a page unchanged, the others appended)."""
+    case = wl("fused-exhaust", 3, 6, 2, 64, "bf16", 8, (30, 30), 4, 0.0, 32)
+    ctx = W.contexts(case)
+    need = int(sum(-(-int(c) // 16) for c in ctx)) * case.num_kv_heads   # prompt pages, all kept
+    snaps, status = [], []
+    for fused in (False, True):
+        run = Run(case, max_pages=need + 1, check_sim=False)
+        try:
+            run.prefill(chunk=64)
+            for step in range(3):   # streams reach 32 tokens: every stream needs a page at once
+                run.decode_step(step, fused=fused)
+            torch.cuda.synchronize()
+            status.append(run.cache.status())
+            snaps.append(run.cache.snapshot())
+        finally:
+            run.close()
+    assert status == [_native.DMS_ERR_POOL_EXHAUSTED] * 2
+    for k in ("n", "pos", "n_pages", "free_list"):
+        np.testing.assert_array_equal(snaps[0][k], snaps[1][k], err_msg=k)
+    assert snaps[0]["free_count"] == snaps[1]["free_count"]
+
+
+def test_fused_step_bad_seq_latches():
+    case = wl("fused-badseq", 2, 4, 1, 64, "bf16", 8, (20, 40), 1, 0.5, 33)
+    run = Run(case, check_sim=False)
+    try:
+        run.prefill(chunk=64)
+        d = lambda x: torch.zeros(x, dtype=torch.bfloat16, device="cuda")
+        ids = torch.tensor([0, 7], dtype=torch.int32, device="cuda")   # 7 >= max_seqs
+        run.cache.decode_step(ids, d((2, 1, 64)), d((2, 1, 64)), torch.zeros((2, 1), dtype=torch.uint8,
+                              device="cuda"), d((2, 4, 64)))
+        torch.cuda.synchronize()
+        assert run.cache.status() == _native.DMS_ERR_BAD_SEQ
+    finally:
+        run.close()
