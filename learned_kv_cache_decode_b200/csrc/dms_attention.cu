@@ -654,7 +654,7 @@ __host__ __device__ inline SmemLayout smem_layout(int ncw, int spw, int stage_by
   L.stages = 0;
   L.bars = ncw * spw * stage_bytes;
   L.misc = L.bars + 8 * ncw * spw;
-  L.merge = L.misc + 128;
+  L.merge = L.misc + 64;
   L.prefix = L.merge + ncw * kMaxGroup * (d + 2) * 4;
   L.sid = L.prefix + (S + 1) * 4;
   L.step = L.sid + S * 4;
@@ -689,9 +689,21 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   constexpr int kMergeThreads = NCW * 32;                  // the consumer warps
   constexpr int kStage = 2 * kPage * D * (int)sizeof(E);   // one page: 16 K rows + 16 V rows
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128-byte TMA swizzle needs 1024-aligned stages. The declaration asks
+  // for that alignment and the launch reserves no slack for rounding up, so a
+  // base that is not aligned would overrun: the CTA then reports and stops
+  // before touching shared memory (uniform over the CTA).
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int spw = a.spw;
   const SmemLayout lay = smem_layout(NCW, spw, kStage, D, a.S, STEP);
+  {
+    uint32_t dyn;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+    if ((uint32_t)(smem - smem_raw) + (uint32_t)lay.total > dyn) {
+      if (threadIdx.x == 0) latch(a.ctrl, DMS_ERR_INVALID);
+      return;
+    }
+  }
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
   // misc: [0] abort, [1] ok, [2] last flag, [3 .. 3+warps) scan scratch, [12] free-stack depth
   // and [13] pages popped by this step (-1: pool exhausted), [14] stream whose combine a split
@@ -1129,7 +1141,7 @@ cudaError_t prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, bo
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&per_sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&per_block_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
-  const int budget = std::min(per_block_smem, per_sm_smem / ctas - 1024) - 1024;   // minus alignment slack
+  const int budget = std::min(per_block_smem, per_sm_smem / ctas - 1024);   // 1 KB per CTA stays reserved
   const int fixed = smem_layout(ncw, 0, stage_bytes, dv.d, dv.S, step).total;
   int spw = std::min(8, (budget - fixed) / (ncw * stage_bytes));
   const int want = env_int("DMS_ATTN_STAGES", 0);
@@ -1142,7 +1154,7 @@ cudaError_t prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, bo
   plan->spw = spw;
   plan->fn = reinterpret_cast<void*>(fn);
   plan->threads = (ncw + (step ? 1 : 0)) * 32;
-  plan->smem = 1024 + (size_t)smem_layout(ncw, spw, stage_bytes, dv.d, dv.S, step).total;
+  plan->smem = (size_t)smem_layout(ncw, spw, stage_bytes, dv.d, dv.S, step).total;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan->smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
