@@ -462,46 +462,76 @@ def main():
     peak, peak_kind = peaks()
     kernel = {"auto": "mma" if tdt == torch.bfloat16 else "simt"}.get(args.attn_kernel, args.attn_kernel)
 
-    # ---- end-to-end pass through the public API with pinned host buffers: per
-    # step one host-to-device copy of each input (every layer appends the same
-    # new token rows) and one device-to-host copy of every layer's output
+    # ---- end-to-end pass through the public API with pinned host buffers. Per
+    # step: one host-to-device copy of each input (every layer appends the same
+    # new token rows) and one device-to-host copy of every layer's output. The
+    # copies run on their own stream, double-buffered, so step t+1's inputs and
+    # step t-1's outputs move while step t computes; events order every reuse.
     e2e = None
     if not args.no_e2e:
         hK, hV, hA, hQ = (to_torch(x, None).pin_memory() for x in (Kd, Vd, Ad, Qd))
-        h_out = torch.empty((L, B, hq, d), dtype=tdt).pin_memory()
-        d_out = torch.empty((L, B, hq, d), dtype=tdt, device=dev)
-        k_, v_ = torch.empty((B, hkv, d), dtype=tdt, device=dev), torch.empty((B, hkv, d), dtype=tdt, device=dev)
-        a_, q_ = torch.empty((B, hkv), dtype=torch.uint8, device=dev), torch.empty((B, hq, d), dtype=tdt, device=dev)
+        h_out = [torch.empty((L, B, hq, d), dtype=tdt).pin_memory() for _ in range(2)]
+        d_out = [torch.empty((L, B, hq, d), dtype=tdt, device=dev) for _ in range(2)]
+        stage = [(torch.empty((B, hkv, d), dtype=tdt, device=dev), torch.empty((B, hkv, d), dtype=tdt, device=dev),
+                  torch.empty((B, hkv), dtype=torch.uint8, device=dev), torch.empty((B, hq, d), dtype=tdt, device=dev))
+                 for _ in range(2)]
+        copy_s = torch.cuda.Stream(device=dev)
+        ev = lambda: torch.cuda.Event()
+        h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
         t0_e2e = t_b + burst_steps
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
+
+        def h2d(t):
+            p = t % 2
+            k_, v_, a_, q_ = stage[p]
+            with torch.cuda.stream(copy_s):
+                if t - 2 >= t0_e2e:
+                    copy_s.wait_event(comp_done[p])   # step t-2 has finished reading this staging set
+                k_.copy_(hK[t], non_blocking=True)
+                v_.copy_(hV[t], non_blocking=True)
+                a_.copy_(hA[t], non_blocking=True)
+                q_.copy_(hQ[t], non_blocking=True)
+                h2d_done[p].record(copy_s)
+
         e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e_a.record(stream)
+        copy_s.wait_stream(stream)
+        h2d(t0_e2e)
         for t in range(t0_e2e, t0_e2e + args.steps):
-            k_.copy_(hK[t], non_blocking=True)
-            v_.copy_(hV[t], non_blocking=True)
-            a_.copy_(hA[t], non_blocking=True)
-            q_.copy_(hQ[t], non_blocking=True)
+            p = t % 2
+            k_, v_, a_, q_ = stage[p]
+            if t + 1 < t0_e2e + args.steps:
+                h2d(t + 1)
+            stream.wait_event(h2d_done[p])
+            if t - 2 >= t0_e2e:
+                stream.wait_event(d2h_done[p])    # step t-2's outputs have left this buffer
             for l in range(L):
                 if fused:
-                    caches[l].decode_step(ids, k_, v_, a_, q_, scale=scale, out=d_out[l])
+                    caches[l].decode_step(ids, k_, v_, a_, q_, scale=scale, out=d_out[p][l])
                 else:
                     caches[l].append(ids, k_, v_, a_)
-                    caches[l].decode_attention(ids, q_, scale=scale, out=d_out[l])
+                    caches[l].decode_attention(ids, q_, scale=scale, out=d_out[p][l])
                 if l == 0:
                     lib.dms_stats(hs[l], sp, None, None, None, pT + t * 16)
-            h_out.copy_(d_out, non_blocking=True)
+            comp_done[p].record(stream)
+            with torch.cuda.stream(copy_s):
+                copy_s.wait_event(comp_done[p])
+                h_out[p].copy_(d_out[p], non_blocking=True)
+                d2h_done[p].record(copy_s)
+        stream.wait_stream(copy_s)
         e_b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e_a.elapsed_time(e_b)
         tot2 = totals.cpu().numpy()[t0_e2e:t0_e2e + args.steps]
         e2e_bytes = float(tot2[:, 1].astype(np.float64).sum()) * L * d * 2 * wl.elem_bytes
         e2e_ms, e2e_bytes = reduce_over_ranks(e2e_ms, e2e_bytes, world, dev)
-        h2d = 2 * row_kv + B * hkv + row_q
-        d2h = L * B * hq * d * wl.elem_bytes
-        e2e = {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
+        h2d_b = 2 * row_kv + B * hkv + row_q
+        d2h_b = L * B * hq * d * wl.elem_bytes
+        e2e = {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d_b,
+               "d2h_bytes_per_step": d2h_b, "ms_per_step": e2e_ms / args.steps,
+               "copies": "own stream, double-buffered (step t+1 in, step t-1 out while step t computes)"}
 
     # ---- CPU baseline: the oracle on a bounded sample of the same step (rank 0, N = 1)
     cpu = None
