@@ -128,6 +128,19 @@ dms_status dms_append(dms_cache* cache, cudaStream_t stream, int32_t n_seqs,
                       const int32_t* seq_ids, const int32_t* cu_tokens, int32_t total_tokens,
                       const void* K, const void* V, const uint8_t* alpha);
 
+/* dms_append with the eviction decisions read from the keys (scope row "alpha
+ * from the logit": paper summary, Method: one neuron of the K projection
+ * per head is repurposed to give the eviction logit; reading R4 of the
+ * design notes: at inference alpha_t = 1 iff that logit is > 0). For every
+ * appended token t and KV head h: alpha = 1 iff K[t, h, alpha_channel] > 0
+ * (zero and NaN keep the token). K and V are stored as given, the logit
+ * channel included. Same bookkeeping and errors as dms_append with those
+ * alpha bits.
+ *   alpha_channel  host int in [0, head_dim) */
+dms_status dms_append_keyed(dms_cache* cache, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                            const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
+                            int32_t alpha_channel);
+
 /* One decode step of GQA attention over the retained tokens (paper summary,
  * Key claims: memory reads dominate decode latency; the mask is never
  * materialised). For each sequence b of the call and query head h:
@@ -166,6 +179,12 @@ dms_status dms_decode_attention(dms_cache* cache, cudaStream_t stream, int32_t n
 dms_status dms_decode_step(dms_cache* cache, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                            const void* K, const void* V, const uint8_t* alpha, const void* Q,
                            int32_t num_q_heads, float scale, void* out, dms_dtype out_dtype);
+
+/* dms_decode_step with the eviction decisions read from the keys, as
+ * dms_append_keyed: alpha = 1 iff K[b, h, alpha_channel] > 0. */
+dms_status dms_decode_step_keyed(dms_cache* cache, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                                 const void* K, const void* V, int32_t alpha_channel, const void* Q,
+                                 int32_t num_q_heads, float scale, void* out, dms_dtype out_dtype);
 
 /* Retained counts and compression ratios (paper summary, Key claims: CR =
  * tokens seen / tokens kept; each head can land at its own CR). Async;

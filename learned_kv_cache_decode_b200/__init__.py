@@ -86,11 +86,17 @@ class DmsCache:
         _native.check(self.lib.dms_seq_reset(self._h, _stream(), int(seq_id)), "dms_seq_reset")
 
     # -- hot path ----------------------------------------------------------
-    def append(self, seq_ids: torch.Tensor, K: torch.Tensor, V: torch.Tensor, alpha: torch.Tensor,
-               cu_tokens: torch.Tensor | None = None) -> None:
-        """Append tokens. seq_ids int32 [B]; K, V [T, Hkv, d]; alpha uint8 [T, Hkv];
-        cu_tokens int32 [B+1] or None for one token per sequence."""
+    def append(self, seq_ids: torch.Tensor, K: torch.Tensor, V: torch.Tensor, alpha: torch.Tensor | None = None,
+               cu_tokens: torch.Tensor | None = None, alpha_channel: int | None = None) -> None:
+        """Append tokens. seq_ids int32 [B]; K, V [T, Hkv, d]; alpha uint8 [T, Hkv], or
+        alpha_channel: alpha = K[..., alpha_channel] > 0; cu_tokens int32 [B+1] or None
+        for one token per sequence."""
         n = int(seq_ids.numel())
+        if alpha_channel is not None:
+            _native.check(self.lib.dms_append_keyed(self._h, _stream(), n, _ptr(seq_ids), _ptr(cu_tokens),
+                                                    int(K.shape[0]), _ptr(K), _ptr(V), int(alpha_channel)),
+                          "dms_append_keyed")
+            return
         _native.check(self.lib.dms_append(self._h, _stream(), n, _ptr(seq_ids), _ptr(cu_tokens),
                                           int(K.shape[0]), _ptr(K), _ptr(V), _ptr(alpha)), "dms_append")
 
@@ -107,16 +113,23 @@ class DmsCache:
                                                     _DTYPES[out.dtype]), "dms_decode_attention")
         return out
 
-    def decode_step(self, seq_ids: torch.Tensor, K: torch.Tensor, V: torch.Tensor, alpha: torch.Tensor,
+    def decode_step(self, seq_ids: torch.Tensor, K: torch.Tensor, V: torch.Tensor, alpha: torch.Tensor | None,
                     Q: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None,
-                    out_dtype: torch.dtype | None = None) -> torch.Tensor:
+                    out_dtype: torch.dtype | None = None, alpha_channel: int | None = None) -> torch.Tensor:
         """One decode step in one launch: append one token per sequence (K, V [B, Hkv, d],
-        alpha uint8 [B, Hkv]) and attend with Q [B, Hq, d] -> out [B, Hq, d]."""
+        alpha uint8 [B, Hkv], or alpha_channel: alpha = K[..., alpha_channel] > 0) and
+        attend with Q [B, Hq, d] -> out [B, Hq, d]."""
         b, hq, d = Q.shape
         if scale is None:
             scale = 1.0 / math.sqrt(d)
         if out is None:
             out = torch.empty((b, hq, d), dtype=out_dtype or Q.dtype, device=Q.device)
+        if alpha_channel is not None:
+            _native.check(self.lib.dms_decode_step_keyed(self._h, _stream(), int(seq_ids.numel()), _ptr(seq_ids),
+                                                         _ptr(K), _ptr(V), int(alpha_channel), _ptr(Q), hq,
+                                                         float(scale), _ptr(out), _DTYPES[out.dtype]),
+                          "dms_decode_step_keyed")
+            return out
         _native.check(self.lib.dms_decode_step(self._h, _stream(), int(seq_ids.numel()), _ptr(seq_ids), _ptr(K),
                                                _ptr(V), _ptr(alpha), _ptr(Q), hq, float(scale), _ptr(out),
                                                _DTYPES[out.dtype]), "dms_decode_step")

@@ -29,7 +29,8 @@ DMS_ATTN_MMA = 2
 
 EXPORTS = ("dms_cache_create", "dms_cache_destroy", "dms_cache_reset", "dms_seq_reset", "dms_append",
            "dms_decode_attention", "dms_stats", "dms_snapshot", "dms_gather_kv", "dms_get_status",
-           "dms_status_string", "dms_launch_count", "dms_decode_attention_noalloc", "dms_decode_step")
+           "dms_status_string", "dms_launch_count", "dms_decode_attention_noalloc", "dms_decode_step",
+           "dms_append_keyed", "dms_decode_step_keyed")
 
 DMS_NOALLOC_MAX_STREAMS = 512
 DMS_NOALLOC_MAX_PIECES = 1024
@@ -111,6 +112,10 @@ def load() -> ctypes.CDLL:
     L.dms_launch_count.restype = i64
     L.dms_decode_step.argtypes = [p, p, i32, p, p, p, p, p, i32, ctypes.c_float, p, ctypes.c_int]
     L.dms_decode_step.restype = st
+    L.dms_append_keyed.argtypes = [p, p, i32, p, p, i32, p, p, i32]
+    L.dms_append_keyed.restype = st
+    L.dms_decode_step_keyed.argtypes = [p, p, i32, p, p, p, i32, p, i32, ctypes.c_float, p, ctypes.c_int]
+    L.dms_decode_step_keyed.restype = st
     L.dms_decode_attention_noalloc.argtypes = [p, ctypes.POINTER(DmsPagedKv), i32, p, p, i32, ctypes.c_float, p,
                                                ctypes.c_int]
     L.dms_decode_attention_noalloc.restype = st

@@ -160,25 +160,69 @@ dms_status dms_seq_reset(dms_cache* h, cudaStream_t stream, int32_t seq_id) {
   return from_cuda(dms::launch_reset_seq(h->dv, stream, seq_id));
 }
 
-dms_status dms_append(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
-                      const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
-                      const uint8_t* alpha) {
+namespace {
+
+dms_status append_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                       const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
+                       const uint8_t* alpha, int32_t alpha_channel) {
   if (!h || n_seqs < 0 || n_seqs > h->cfg.max_seqs || total_tokens < 0) return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
+  if (alpha_channel >= h->cfg.head_dim) return DMS_ERR_INVALID;
   if (n_seqs == 0) return DMS_OK;
-  if (!seq_ids || (total_tokens > 0 && (!K || !V || !alpha))) return DMS_ERR_INVALID;
+  if (!seq_ids || (total_tokens > 0 && (!K || !V || (alpha_channel < 0 && !alpha)))) return DMS_ERR_INVALID;
   if (!aligned16(K) || !aligned16(V)) return DMS_ERR_INVALID;
   int launches = 0;
   cudaError_t e;
   if (cu_tokens == nullptr) {
     if (total_tokens != n_seqs) return DMS_ERR_INVALID;
-    e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, &launches);
+    e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, &launches);
   } else {
     e = dms::launch_append_bulk(h->dv, stream, n_seqs, seq_ids, cu_tokens, total_tokens, K, V, alpha,
-                                &launches);
+                                alpha_channel, &launches);
   }
   h->launches += launches;
   return from_cuda(e);
+}
+
+dms_status step_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids, const void* K,
+                     const void* V, const uint8_t* alpha, int32_t alpha_channel, const void* Q, int32_t num_q_heads,
+                     float scale, void* out, dms_dtype out_dtype) {
+  if (!h || n_seqs < 0 || n_seqs > h->cfg.max_seqs) return DMS_ERR_INVALID;
+  if (dms_status s = check_usable(h)) return s;
+  if (num_q_heads < h->cfg.num_kv_heads || num_q_heads % h->cfg.num_kv_heads != 0) return DMS_ERR_INVALID;
+  if (num_q_heads / h->cfg.num_kv_heads > dms::kMaxGroup) return DMS_ERR_INVALID;
+  if (out_dtype != DMS_BF16 && out_dtype != DMS_F32) return DMS_ERR_INVALID;
+  if (alpha_channel >= h->cfg.head_dim) return DMS_ERR_INVALID;
+  if (n_seqs == 0) return DMS_OK;
+  if (!seq_ids || !K || !V || (alpha_channel < 0 && !alpha) || !Q || !out) return DMS_ERR_INVALID;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(out)) return DMS_ERR_INVALID;
+  if (!h->has_step) {
+    int launches = 0;
+    cudaError_t e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, &launches);
+    h->launches += launches;
+    if (e != cudaSuccess) return DMS_ERR_CUDA;
+    h->launches += 1;
+    return from_cuda(dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
+                                           out_dtype == DMS_F32));
+  }
+  h->launches += 1;
+  return from_cuda(dms::launch_step(h->dv, h->step_plan, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, Q,
+                                    num_q_heads, scale, out, out_dtype == DMS_F32));
+}
+
+}  // namespace
+
+dms_status dms_append(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                      const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
+                      const uint8_t* alpha) {
+  return append_impl(h, stream, n_seqs, seq_ids, cu_tokens, total_tokens, K, V, alpha, -1);
+}
+
+dms_status dms_append_keyed(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                            const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
+                            int32_t alpha_channel) {
+  if (alpha_channel < 0) return DMS_ERR_INVALID;
+  return append_impl(h, stream, n_seqs, seq_ids, cu_tokens, total_tokens, K, V, nullptr, alpha_channel);
 }
 
 dms_status dms_decode_attention(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
@@ -199,26 +243,14 @@ dms_status dms_decode_attention(dms_cache* h, cudaStream_t stream, int32_t n_seq
 dms_status dms_decode_step(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                            const void* K, const void* V, const uint8_t* alpha, const void* Q, int32_t num_q_heads,
                            float scale, void* out, dms_dtype out_dtype) {
-  if (!h || n_seqs < 0 || n_seqs > h->cfg.max_seqs) return DMS_ERR_INVALID;
-  if (dms_status s = check_usable(h)) return s;
-  if (num_q_heads < h->cfg.num_kv_heads || num_q_heads % h->cfg.num_kv_heads != 0) return DMS_ERR_INVALID;
-  if (num_q_heads / h->cfg.num_kv_heads > dms::kMaxGroup) return DMS_ERR_INVALID;
-  if (out_dtype != DMS_BF16 && out_dtype != DMS_F32) return DMS_ERR_INVALID;
-  if (n_seqs == 0) return DMS_OK;
-  if (!seq_ids || !K || !V || !alpha || !Q || !out) return DMS_ERR_INVALID;
-  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(out)) return DMS_ERR_INVALID;
-  if (!h->has_step) {
-    int launches = 0;
-    cudaError_t e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, &launches);
-    h->launches += launches;
-    if (e != cudaSuccess) return DMS_ERR_CUDA;
-    h->launches += 1;
-    return from_cuda(dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
-                                           out_dtype == DMS_F32));
-  }
-  h->launches += 1;
-  return from_cuda(dms::launch_step(h->dv, h->step_plan, stream, n_seqs, seq_ids, K, V, alpha, Q, num_q_heads,
-                                    scale, out, out_dtype == DMS_F32));
+  return step_impl(h, stream, n_seqs, seq_ids, K, V, alpha, -1, Q, num_q_heads, scale, out, out_dtype);
+}
+
+dms_status dms_decode_step_keyed(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                                 const void* K, const void* V, int32_t alpha_channel, const void* Q,
+                                 int32_t num_q_heads, float scale, void* out, dms_dtype out_dtype) {
+  if (alpha_channel < 0) return DMS_ERR_INVALID;
+  return step_impl(h, stream, n_seqs, seq_ids, K, V, nullptr, alpha_channel, Q, num_q_heads, scale, out, out_dtype);
 }
 
 dms_status dms_stats(dms_cache* h, cudaStream_t stream, int32_t* retained, int32_t* seen, float* head_cr,

@@ -49,8 +49,7 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
-                     const uint8_t* __restrict__ K, const uint8_t* __restrict__ V,
-                     const uint8_t* __restrict__ alpha) {
+                     const uint8_t* __restrict__ K, const uint8_t* __restrict__ V, const AlphaSrc asrc) {
   extern __shared__ int s_phys[];   // [nst] physical slot that receives each stream's rows, -1 none
   __shared__ int s_warp[kDecodeThreads / 32];
   constexpr int T = kDecodeThreads;
@@ -83,7 +82,7 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     al = 0;
     if (i < nst) {
       seq = __ldg(seq_ids + i / dv.hkv);
-      al = __ldg(alpha + i) != 0;
+      al = alpha_at(asrc, (size_t)(i / dv.hkv), i % dv.hkv);
     }
   };
   int seq, al;
@@ -202,7 +201,7 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
 // marked.
 __global__ void __launch_bounds__(256)
 bulk_count_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
-                  const int32_t* __restrict__ cu, int total_tokens, const uint8_t* __restrict__ alpha) {
+                  const int32_t* __restrict__ cu, int total_tokens, const AlphaSrc asrc) {
   __shared__ int s_warp[8];
   const int i = blockIdx.x;
   if (read_status(dv.ctrl) != 0) return;
@@ -225,7 +224,7 @@ bulk_count_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     int marked = 0;
     if (j >= dv.w) {
       const int jp = j - dv.w;
-      marked = (jp >= s0) ? (alpha[(size_t)(t0 + jp - s0) * dv.hkv + kvh] != 0)
+      marked = (jp >= s0) ? alpha_at(asrc, (size_t)(t0 + jp - s0), kvh)
                           : (dv.ring[(size_t)st * dv.w + jp % dv.w] & 1);
     }
     fresh += !marked;
@@ -283,7 +282,7 @@ bulk_pages_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids) {
 __global__ void __launch_bounds__(256)
 bulk_write_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
                   const int32_t* __restrict__ cu, const uint8_t* __restrict__ K,
-                  const uint8_t* __restrict__ V, const uint8_t* __restrict__ alpha) {
+                  const uint8_t* __restrict__ V, const AlphaSrc asrc) {
   __shared__ int s_warp[8];
   __shared__ int s_phys[256];
   if (read_status(dv.ctrl) != 0) return;
@@ -315,7 +314,7 @@ bulk_write_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     int phys = -1;
     if (active) {
       const int slot = retire ? (r >> 1) : n_cur + pre;
-      const int a = alpha[(size_t)(t0 + t) * dv.hkv + kvh] != 0;
+      const int a = alpha_at(asrc, (size_t)(t0 + t), kvh);
       ring[j % dv.w] = (slot << 1) | a;
       const bool dead = a && (j + dv.w <= s_last);
       const int page = slot / kPage < dv.mps ? pt[slot / kPage] : -1;
@@ -475,23 +474,26 @@ cudaError_t launch_init_state(const Dev& dv, cudaStream_t st) {
 }
 
 cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
-                                 const void* K, const void* V, const uint8_t* alpha, int* launches) {
+                                 const void* K, const void* V, const uint8_t* alpha, int alpha_channel,
+                                 int* launches) {
+  const AlphaSrc asrc{alpha, (const uint8_t*)K, alpha_channel, dv.hkv, dv.d, dv.elem_bytes};
   const int nst = n_seqs * dv.hkv;
   if (nst == 0) return cudaSuccess;
   *launches += 1;
   return launch_dependent(append_decode_kernel, dim3(1), dim3(kDecodeThreads), (size_t)nst * sizeof(int), st, dv,
-                          n_seqs, seq_ids, (const uint8_t*)K, (const uint8_t*)V, alpha);
+                          n_seqs, seq_ids, (const uint8_t*)K, (const uint8_t*)V, asrc);
 }
 
 cudaError_t launch_append_bulk(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
                                const int32_t* cu_tokens, int total_tokens, const void* K, const void* V,
-                               const uint8_t* alpha, int* launches) {
+                               const uint8_t* alpha, int alpha_channel, int* launches) {
+  const AlphaSrc asrc{alpha, (const uint8_t*)K, alpha_channel, dv.hkv, dv.d, dv.elem_bytes};
   const int nst = n_seqs * dv.hkv;
   if (nst == 0) return cudaSuccess;
-  bulk_count_kernel<<<nst, 256, 0, st>>>(dv, n_seqs, seq_ids, cu_tokens, total_tokens, alpha);
+  bulk_count_kernel<<<nst, 256, 0, st>>>(dv, n_seqs, seq_ids, cu_tokens, total_tokens, asrc);
   bulk_pages_kernel<<<1, 256, 0, st>>>(dv, n_seqs, seq_ids);
   bulk_write_kernel<<<nst, 256, 0, st>>>(dv, n_seqs, seq_ids, cu_tokens, (const uint8_t*)K,
-                                        (const uint8_t*)V, alpha);
+                                        (const uint8_t*)V, asrc);
   *launches += 3;
   return cudaGetLastError();
 }

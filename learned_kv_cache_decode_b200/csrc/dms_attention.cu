@@ -49,7 +49,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct StepArgs {
   const uint8_t* K;       // [n_seqs][hkv][d] new key rows
   const uint8_t* V;       // [n_seqs][hkv][d] new value rows
-  const uint8_t* alpha;   // [n_seqs][hkv] eviction decisions of the new tokens
+  AlphaSrc asrc;          // eviction decisions of the new tokens
   Dev dv;                 // the cache, writable
 };
 
@@ -749,7 +749,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     int local = 0;
     for (int i = b0; i < e0; ++i) {
       const int seq = a.seq_ids[i / a.hkv];
-      const int al = STEP ? a.step.alpha[i] : 0;   // same round trip as the seq id
+      const int al = STEP ? alpha_at(a.step.asrc, (size_t)(i / a.hkv), i % a.hkv) : 0;   // same round trip as the seq id
       int pages = 0, st = 0;
       if (seq < 0 || seq >= a.max_seqs) {
         if constexpr (STEP) s_flag[i] = 4;   // latched once every CTA has read the status
@@ -1237,13 +1237,13 @@ cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t s
 }
 
 cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
-                        const void* K, const void* V, const uint8_t* alpha, const void* Q, int hq, float scale,
-                        void* out, int out_f32) {
+                        const void* K, const void* V, const uint8_t* alpha, int alpha_channel, const void* Q, int hq,
+                        float scale, void* out, int out_f32) {
   if (n_seqs == 0) return cudaSuccess;
   AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32);
   a.step.K = (const uint8_t*)K;
   a.step.V = (const uint8_t*)V;
-  a.step.alpha = alpha;
+  a.step.asrc = AlphaSrc{alpha, (const uint8_t*)K, alpha_channel, dv.hkv, dv.d, dv.elem_bytes};
   a.step.dv = dv;
   return launch_dependent(reinterpret_cast<KernelFn>(plan.fn), dim3(plan.grid), dim3(plan.threads), plan.smem, st,
                           a, plan.tmap);

@@ -16,6 +16,26 @@ constexpr int kMaxGroup = 8;       // query heads per KV head handled by one ker
 constexpr int kMaxStreams = 8192;  // max_seqs * num_kv_heads
 constexpr int kMaxKvHeads = 256;
 
+// Where the eviction decisions of appended tokens come from: an explicit
+// uint8 array [rows][hkv] (channel < 0), or the sign of one designated
+// channel of each token's key row: alpha = 1 iff K[row][kvh][channel] > 0
+// (the eviction logit read from a repurposed key neuron; zero and NaN keep
+// the token).
+struct AlphaSrc {
+  const uint8_t* alpha;   // [rows][hkv] when channel < 0
+  const uint8_t* K;       // [rows][hkv][d] elements
+  int channel, hkv, d, elem_bytes;
+};
+
+__device__ __forceinline__ int alpha_at(const AlphaSrc& s, size_t row, int kvh) {
+  if (s.channel < 0) return s.alpha[row * s.hkv + kvh] != 0;
+  const size_t e = (row * s.hkv + kvh) * (size_t)s.d + s.channel;
+  const float logit = s.elem_bytes == 2
+                          ? __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(s.K)[e] << 16)
+                          : reinterpret_cast<const float*>(s.K)[e];
+  return logit > 0.f;
+}
+
 // Control words (device int32).
 enum : int {
   kCtrlStatus = 0,   // latched dms_status, 0 = healthy
@@ -287,10 +307,11 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
 cudaError_t prepare_aux_kernels();
 cudaError_t launch_init_state(const Dev& dv, cudaStream_t st);
 cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
-                                 const void* K, const void* V, const uint8_t* alpha, int* launches);
+                                 const void* K, const void* V, const uint8_t* alpha, int alpha_channel,
+                                 int* launches);
 cudaError_t launch_append_bulk(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
                                const int32_t* cu_tokens, int total_tokens, const void* K, const void* V,
-                               const uint8_t* alpha, int* launches);
+                               const uint8_t* alpha, int alpha_channel, int* launches);
 cudaError_t launch_reset_seq(const Dev& dv, cudaStream_t st, int seq);
 cudaError_t launch_stats(const Dev& dv, cudaStream_t st, int32_t* retained, int32_t* seen, float* head_cr,
                          int64_t* totals);
@@ -313,8 +334,8 @@ cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int n
 // The fused decode step (append + attention in one launch); see dms_decode_step.
 cudaError_t step_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan);
 cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
-                        const void* K, const void* V, const uint8_t* alpha, const void* Q, int hq, float scale,
-                        void* out, int out_f32);
+                        const void* K, const void* V, const uint8_t* alpha, int alpha_channel, const void* Q, int hq,
+                        float scale, void* out, int out_f32);
 constexpr int kStepMaxStreams = 1024;   // caches with more streams run the step as two launches
 
 cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,

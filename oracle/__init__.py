@@ -80,6 +80,20 @@ def retained_count_closed_form(alpha_seq, s: int, window: int) -> int:
 # ---------------------------------------------------------------------------
 # Attention
 
+def alpha_from_keys(K: np.ndarray, channel: int) -> np.ndarray:
+    """Eviction decisions read from a designated key channel: uint8 [..., Hkv].
+
+    Method section of the paper summary: one neuron of the K projection per head
+    is repurposed to produce the eviction logit. At inference (reading R4) the
+    token is marked iff that logit is > 0; zero and NaN keep it. K holds stored
+    values: bf16 bits as uint16, or float32.
+    """
+    x = np.asarray(K)
+    logit = (x[..., channel].astype(np.uint32) << np.uint32(16)).view(np.float32) if x.dtype == np.uint16 \
+        else x[..., channel].astype(np.float32)
+    return (logit > 0).astype(np.uint8)
+
+
 def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, alpha_seq: np.ndarray,
               window: int, scale: float) -> np.ndarray:
     """Masked softmax attention of g query heads over one stream, fp64.

@@ -39,8 +39,12 @@ class Run:
     """One workload on one cache plus its oracle simulator, call for call."""
 
     def __init__(self, wl: W.Workload, attn_kernel: str = "auto", steps: int | None = None,
-                 max_pages: int | None = None, check_sim: bool = True):
+                 max_pages: int | None = None, check_sim: bool = True, alpha_channel: int | None = None):
+        """alpha_channel: the library reads every token's alpha from the sign of this key
+        channel (dms_append_keyed / dms_decode_step_keyed); the oracle gets the same bits
+        from oracle.alpha_from_keys."""
         self.wl = wl
+        self.alpha_channel = alpha_channel
         self.ctx = W.contexts(wl)
         self.steps = wl.decode_steps if steps is None else steps
         mp, mps = pool_pages(wl, self.ctx, self.steps)
@@ -69,16 +73,25 @@ class Run:
                 counts.append(t)
                 Ks.append(K)
                 Vs.append(V)
-                As.append(W.alpha(self.wl, b, int(self.seen[b]), t))
+                As.append(self.alpha_of(b, int(self.seen[b]), t, K))
             if not ids:
                 return
             self.append_bulk(ids, counts, np.concatenate(Ks), np.concatenate(Vs), np.concatenate(As))
 
+    def alpha_of(self, b: int, start: int, count: int, K: np.ndarray | None = None) -> np.ndarray:
+        """Eviction bits of positions [start, start+count) of sequence b."""
+        if self.alpha_channel is None:
+            return W.alpha(self.wl, b, start, count)
+        if K is None:
+            K, _ = W.kv(self.wl, b, start, count)
+        return oracle.alpha_from_keys(K, self.alpha_channel)
+
     def append_bulk(self, ids, counts, K, V, A) -> None:
         cu = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        alpha = None if self.alpha_channel is not None else torch.from_numpy(np.ascontiguousarray(A)).cuda()
         self.cache.append(torch.tensor(ids, dtype=torch.int32, device="cuda"), to_device(K, self.wl),
-                          to_device(V, self.wl), torch.from_numpy(np.ascontiguousarray(A)).cuda(),
-                          cu_tokens=torch.from_numpy(cu).cuda())
+                          to_device(V, self.wl), alpha, cu_tokens=torch.from_numpy(cu).cuda(),
+                          alpha_channel=self.alpha_channel)
         if self.sim is not None:
             rc, _ = self.sim.append(ids, counts, A)
             assert rc == 0, rc
@@ -90,7 +103,7 @@ class Run:
         e = self._blk.get(b)
         if e is None or not (e[0] <= pos < e[0] + len(e[3])):
             K, V = W.kv(self.wl, b, pos, block, threads=1)
-            e = (pos, K, V, W.alpha(self.wl, b, pos, block))
+            e = (pos, K, V, self.alpha_of(b, pos, block, K))
             self._blk[b] = e
         o = pos - e[0]
         return e[1][o], e[2][o], e[3][o]
@@ -110,17 +123,19 @@ class Run:
         seqs = list(range(self.wl.batch)) if seqs is None else list(seqs)
         K, V, A, Q = self.decode_inputs(step, seqs)
         ids = torch.tensor(seqs, dtype=torch.int32, device="cuda")
+        dev_alpha = None if self.alpha_channel is not None else torch.from_numpy(A).cuda()
         if fused:
-            out = self.cache.decode_step(ids, to_device(K, self.wl), to_device(V, self.wl),
-                                         torch.from_numpy(A).cuda(), to_device(Q, self.wl), scale=self.scale,
-                                         out_dtype=out_dtype)
+            out = self.cache.decode_step(ids, to_device(K, self.wl), to_device(V, self.wl), dev_alpha,
+                                         to_device(Q, self.wl), scale=self.scale, out_dtype=out_dtype,
+                                         alpha_channel=self.alpha_channel)
             if self.sim is not None:
                 rc, _ = self.sim.append(seqs, [1] * len(seqs), A)
                 assert rc == 0, rc
             for b in seqs:
                 self.seen[b] += 1
             return out, Q
-        self.cache.append(ids, to_device(K, self.wl), to_device(V, self.wl), torch.from_numpy(A).cuda())
+        self.cache.append(ids, to_device(K, self.wl), to_device(V, self.wl), dev_alpha,
+                          alpha_channel=self.alpha_channel)
         if self.sim is not None:
             rc, _ = self.sim.append(seqs, [1] * len(seqs), A)
             assert rc == 0, rc
@@ -134,7 +149,7 @@ class Run:
         """Oracle output [Hq, d] for sequence b at its current last position."""
         T = int(self.seen[b])
         K, V = W.kv(self.wl, b, 0, T)
-        A = W.alpha(self.wl, b, 0, T)
+        A = self.alpha_of(b, 0, T, K)
         return oracle.decode_gqa(W.to_f64(q), W.to_f64(K), W.to_f64(V), A, self.wl.window, self.scale)
 
     def check_metadata(self) -> None:

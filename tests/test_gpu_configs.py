@@ -65,9 +65,11 @@ def test_qwen_r1_32b_chains():
     _run_config("qwen-r1-32b-chains", check_steps={0, 255}, check_seqs=[0, 21, 63], metadata_every=128)
 
 
-def test_longrun_2k_30k():
+@pytest.mark.parametrize("fused", [False, True], ids=["two_launches", "fused_step"])
+def test_longrun_2k_30k(fused):
     """2K prompt then 30K decode steps; slot reuse, page-table growth and sequence
-    restarts (page returns and re-pops) checked against the oracle every 1K steps."""
+    restarts (page returns and re-pops) checked against the oracle every 1K steps,
+    through dms_append + dms_decode_attention or through dms_decode_step."""
     wl = W.WORKLOADS["longrun-2k-30k"]
     run = Run(wl)
     try:
@@ -83,7 +85,7 @@ def test_longrun_2k_30k():
                 run._blk.pop(b, None)
                 run.ctx[b] = 1024
                 run.prefill(chunk=1024, seqs=[b])
-            out, Q = run.decode_step(step)
+            out, Q = run.decode_step(step, fused=fused)
             if (step + 1) % 1000 == 0:
                 torch.cuda.synchronize()
                 run.check_metadata()

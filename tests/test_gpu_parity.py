@@ -304,3 +304,54 @@ def test_fused_step_bad_seq_latches():
         assert run.cache.status() == _native.DMS_ERR_BAD_SEQ
     finally:
         run.close()
+
+
+# ---------------------------------------------------------------------------
+# alpha read from a designated key channel (dms_append_keyed, dms_decode_step_keyed)
+
+KEYED = [
+    (wl("keyed-bf16-g7-d128", 3, 21, 3, 128, "bf16", 16, (1, 700), 6, 0.5, 41), 5),
+    (wl("keyed-bf16-g4-d64-w1", 2, 8, 2, 64, "bf16", 1, (20, 300), 5, 0.5, 42), 63),
+    (wl("keyed-f32-g4-d64", 2, 8, 2, 64, "f32", 24, (1, 400), 5, 0.5, 43), 0),
+]
+
+
+@pytest.mark.parametrize("case,channel", KEYED, ids=[c.name for c, _ in KEYED])
+@pytest.mark.parametrize("fused", [False, True], ids=["two_launches", "fused_step"])
+def test_alpha_from_key_channel(case, channel, fused):
+    """The library reads alpha from the sign of key channel `channel` (prefill and every
+    decode step); the oracle gets the same bits from oracle.alpha_from_keys. Metadata bit
+    for bit, outputs within tolerance."""
+    run = Run(case, alpha_channel=channel)
+    try:
+        run.prefill(chunk=97)
+        run.check_metadata()
+        for step in range(case.decode_steps):
+            out, Q = run.decode_step(step, fused=fused)
+            torch.cuda.synchronize()
+            for b in range(case.batch):
+                tol = dict(max_abs=1e-4, mean_abs=1e-5) if case.dtype == "f32" else {}
+                compare(out[b], run.oracle_out(b, Q[b]), **tol)
+            run.check_metadata()
+        snap = run.sim.snapshot()
+        assert 0 < int(snap["n"].sum()) < int(run.seen.sum()) * case.num_kv_heads   # some tokens did leave
+        assert run.cache.status() == _native.DMS_OK
+    finally:
+        run.close()
+
+
+def test_keyed_entry_points_reject_a_channel_outside_head_dim():
+    case = wl("keyed-bad", 1, 2, 1, 64, "bf16", 8, (10, 10), 1, 0.5, 44)
+    run = Run(case, check_sim=False)
+    try:
+        ids = torch.zeros(1, dtype=torch.int32, device="cuda")
+        K = torch.zeros((1, 1, 64), dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(_native.DmsError) as e:
+            run.cache.append(ids, K, K, None, alpha_channel=64)
+        assert e.value.code == _native.DMS_ERR_INVALID
+        with pytest.raises(_native.DmsError) as e:
+            run.cache.decode_step(ids, K, K, None, torch.zeros((1, 2, 64), dtype=torch.bfloat16, device="cuda"),
+                                  alpha_channel=-1 + 65)
+        assert e.value.code == _native.DMS_ERR_INVALID
+    finally:
+        run.close()

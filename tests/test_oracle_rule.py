@@ -8,7 +8,9 @@ What pins what:
   * brute force over every alpha pattern of length <= 12 compares the
     simulator (ring-free lookup, slot reuse) with the visibility definition;
   * a hand-derived free-stack trace (tests/golden/page_pops.txt) fixes the
-    page-pop and reset order.
+    page-pop and reset order;
+  * hand-encoded logits (tests/golden/alpha_from_keys.txt) fix the sign rule
+    that reads alpha from a designated key channel (zero and NaN keep).
 """
 import os
 import itertools
@@ -201,3 +203,47 @@ def test_pool_exhaustion_and_stream_capacity():
     sim2 = oracle.Sim(1, 1, 8, max_pages=8, max_pages_per_stream=1)
     assert sim2.append([0], [16], np.zeros((16, 1), np.uint8))[0] == 0
     assert sim2.append([0], [1], np.zeros((1, 1), np.uint8))[0] == 6
+
+
+# ---------------------------------------------------------------------------
+# alpha read from a designated key channel (the eviction logit)
+
+def _golden_logits():
+    rows = []
+    for line in open(os.path.join(GOLD, "alpha_from_keys.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        dt, bits, want = line.split()
+        rows.append((dt, int(bits, 16), int(want)))
+    return rows
+
+
+def test_golden_alpha_from_keys():
+    rows = _golden_logits()
+    assert len(rows) >= 10
+    for dt, bits, want in rows:
+        d = 8
+        if dt == "bf16":
+            K = np.zeros((1, 2, d), dtype=np.uint16)
+            K[0, 1, 5] = bits
+        else:
+            K = np.zeros((1, 2, d), dtype=np.float32)
+            K.view(np.uint32)[0, 1, 5] = bits
+        a = oracle.alpha_from_keys(K, 5)
+        assert a.shape == (1, 2) and a.dtype == np.uint8
+        assert a[0, 1] == want, (dt, hex(bits))
+        assert a[0, 0] == 0   # the other head's channel holds +0.0
+
+
+def test_alpha_from_keys_reads_only_the_designated_channel():
+    rng = np.random.default_rng(5)
+    K = rng.standard_normal((50, 3, 16)).astype(np.float32)
+    for c in (0, 7, 15):
+        a = oracle.alpha_from_keys(K, c)
+        K2 = K.copy()
+        K2[..., [x for x in range(16) if x != c]] *= -1.0   # other channels do not matter
+        np.testing.assert_array_equal(oracle.alpha_from_keys(K2, c), a)
+        K3 = K.copy()
+        K3[..., c] *= -1.0   # flipping the logit flips every non-zero decision
+        np.testing.assert_array_equal(oracle.alpha_from_keys(K3, c), 1 - a)
