@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--workload", default="qwen-r1-7b-32k", choices=sorted(W.WORKLOADS))
     ap.add_argument("--layers", type=int, default=0, help="layer caches per step (0: enough to exceed 8x L2)")
     ap.add_argument("--attn-kernel", default="auto", choices=["auto", "mma", "simt"])
+    ap.add_argument("--window", type=int, default=0,
+                    help="override the workload's delayed-eviction window w (1 = immediate eviction)")
     ap.add_argument("--step", default="fused", choices=["fused", "separate"],
                     help="fused: one dms_decode_step launch per layer; separate: dms_append + dms_decode_attention")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
@@ -287,6 +289,9 @@ def run_reference(args, wl, world, rank):
 def main():
     args = parse_args()
     wl = W.WORKLOADS[args.workload]
+    if args.window:
+        import dataclasses
+        wl = dataclasses.replace(wl, window=args.window)
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         run_reference(args, wl, world, rank)
