@@ -17,6 +17,7 @@ struct dms_cache {
   dms::AttnPlan plan{};
   dms::AttnPlan step_plan{};   // fused decode step (append + attention in one launch)
   bool has_step = false;       // else dms_decode_step issues the two launches
+  uint64_t step_launches = 0;  // fused steps launched since the counters were last cleared
   int64_t launches = 0;
   bool poisoned = false;   // a device error was observed by dms_get_status
 };
@@ -147,9 +148,12 @@ dms_status dms_cache_reset(dms_cache* h, cudaStream_t stream) {
   if (!h) return DMS_ERR_INVALID;
   if (dms_status s = check_device(h)) return s;
   cudaError_t e = cudaMemsetAsync(h->dv.page_table, 0xff, (size_t)h->dv.S * h->dv.mps * sizeof(int32_t), stream);
-  if (e == cudaSuccess) e = dms::launch_init_state(h->dv, stream);
+  if (e == cudaSuccess) e = dms::launch_init_state(h->dv, stream);   // clears the step counter too
   h->launches += 1;
-  if (e == cudaSuccess) h->poisoned = false;
+  if (e == cudaSuccess) {
+    h->poisoned = false;
+    h->step_launches = 0;
+  }
   return from_cuda(e);
 }
 
@@ -206,8 +210,10 @@ dms_status step_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const in
                                            out_dtype == DMS_F32));
   }
   h->launches += 1;
-  return from_cuda(dms::launch_step(h->dv, h->step_plan, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, Q,
-                                    num_q_heads, scale, out, out_dtype == DMS_F32));
+  const cudaError_t e = dms::launch_step(h->dv, h->step_plan, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, Q,
+                                         num_q_heads, scale, out, out_dtype == DMS_F32, h->step_launches);
+  if (e == cudaSuccess) h->step_launches += 1;
+  return from_cuda(e);
 }
 
 }  // namespace

@@ -50,6 +50,7 @@ struct StepArgs {
   const uint8_t* K;       // [n_seqs][hkv][d] new key rows
   const uint8_t* V;       // [n_seqs][hkv][d] new value rows
   AlphaSrc asrc;          // eviction decisions of the new tokens
+  unsigned long long launch_index;   // fused steps launched on this cache before this one
   Dev dv;                 // the cache, writable
 };
 
@@ -457,18 +458,38 @@ __device__ __forceinline__ void load4<uint16_t>(const uint16_t* p, float (&x)[4]
 // fp32 from the stored inputs, scaled into base 2 like the page scores.
 // Warp-collective: the D/4 lanes of one head reduce the dot product, so
 // every lane of the warp calls it, `use` or not.
+// The inputs of the new token's term for one merge item: q, k and v at dims
+// [4 d4, 4 d4 + 4) of query head h and its stream i.
+struct NewTok {
+  float q[4], k[4], v[4];
+};
+
+template <int D, typename E>
+__device__ __forceinline__ void fetch_new_token(const AttnArgs& a, int i, int h, int d4, NewTok& t) {
+  const int b = i / a.hkv, kvh = i % a.hkv;
+  load4<E>(reinterpret_cast<const E*>(a.Q) + ((size_t)b * a.hq + (size_t)kvh * a.g + h) * D + 4 * d4, t.q);
+  load4<E>(reinterpret_cast<const E*>(a.step.K) + (size_t)i * D + 4 * d4, t.k);
+  load4<E>(reinterpret_cast<const E*>(a.step.V) + (size_t)i * D + 4 * d4, t.v);
+}
+
+// Merge the new token (score q . k in fp32, scaled into base 2 like the page
+// scores; value v) into (M, L, O) when `use`. Warp-collective: the D/4 lanes
+// of one head reduce the dot product, so every lane of the warp calls it.
+template <int D>
+__device__ __forceinline__ void apply_new_token(const NewTok& t, float sl2e, bool use, float& M, float& L,
+                                                float4& O) {
+  float dot = t.q[0] * t.k[0] + t.q[1] * t.k[1] + t.q[2] * t.k[2] + t.q[3] * t.k[3];
+#pragma unroll
+  for (int o = D / 8; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  if (use) merge_into(M, L, O, dot * sl2e, 1.f, make_float4(t.v[0], t.v[1], t.v[2], t.v[3]));
+}
+
 template <int D, typename E>
 __device__ __forceinline__ void add_new_token(const AttnArgs& a, int i, int h, int d4, bool use, float& M,
                                               float& L, float4& O) {
-  const int b = i / a.hkv, kvh = i % a.hkv;
-  float q4[4], k4[4], v4[4];
-  load4<E>(reinterpret_cast<const E*>(a.Q) + ((size_t)b * a.hq + (size_t)kvh * a.g + h) * D + 4 * d4, q4);
-  load4<E>(reinterpret_cast<const E*>(a.step.K) + (size_t)i * D + 4 * d4, k4);
-  load4<E>(reinterpret_cast<const E*>(a.step.V) + (size_t)i * D + 4 * d4, v4);
-  float dot = q4[0] * k4[0] + q4[1] * k4[1] + q4[2] * k4[2] + q4[3] * k4[3];
-#pragma unroll
-  for (int o = D / 8; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-  if (use) merge_into(M, L, O, dot * a.sl2e, 1.f, make_float4(v4[0], v4[1], v4[2], v4[3]));
+  NewTok t;
+  fetch_new_token<D, E>(a, i, h, d4, t);
+  apply_new_token<D>(t, a.sl2e, use, M, L, O);
 }
 
 // Combine the partials first .. last of stream i into its output, items
@@ -525,7 +546,7 @@ template <int D, typename E>
 __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int* prefix, const int* sid,
                                        const int* s_nold, const int* s_pos, int* s_rslot, int* s_tslot,
                                        int* s_flag, int* s_rank, int* misc, bool healthy,
-                                       volatile int* abort_flag) {
+                                       volatile int* abort_flag, int K0, int K1) {
   const int lane = threadIdx.x & 31;
   const Dev& dv = a.step.dv;
   // Wait (no spinning) until the consumer warps have resolved every stream's
@@ -580,10 +601,33 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
     *reinterpret_cast<volatile int*>(&misc[15]) = 1;   // the consumers may read the decisions
     // This CTA is done reading the pre-step state (its reads were ordered
     // before this point by the plan's barriers and barrier 2).
-    red_add_release_gpu(&a.ctrl[kCtrlPlanned], 1);
+    red_add_release_gpu_u64(reinterpret_cast<unsigned long long*>(&a.ctrl[kCtrlPlanned]), 1ull);
   }
   __syncwarp();
   if (!healthy) return;
+
+  // The streams whose outputs this CTA may produce (whole pieces, and the
+  // range's last piece, which it may combine) merge their new token at the
+  // end of the piece: pull its query rows and new K and V rows into L2 while
+  // the pages stream, one prefetch per 128-byte line.
+  for (int k = K0; k < K1;) {
+    const int i = stream_of(prefix, nst, k);
+    const int pe = min(prefix[i + 1], K1);
+    if (prefix[i] >= K0 || pe == K1) {
+      const int b = i / a.hkv, kvh = i % a.hkv;
+      const int qlines = a.g * D * (int)sizeof(E) / 128, rlines = D * (int)sizeof(E) / 128;
+      const uint8_t* qrow = a.Q + ((size_t)b * a.hq + (size_t)kvh * a.g) * D * sizeof(E);
+      const uint8_t* krow = a.step.K + (size_t)i * D * sizeof(E);
+      const uint8_t* vrow = a.step.V + (size_t)i * D * sizeof(E);
+      for (int l = lane; l < qlines + 2 * rlines; l += 32) {
+        const uint8_t* p = l < qlines ? qrow + (size_t)l * 128
+                                      : (l < qlines + rlines ? krow + (size_t)(l - qlines) * 128
+                                                             : vrow + (size_t)(l - qlines - rlines) * 128);
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+      }
+    }
+    k = pe;
+  }
 
   const int G = gridDim.x;
   // Streams with nothing retained before the step attend to the new token alone.
@@ -601,7 +645,10 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
 
   // Wait until every CTA has read the pre-step state, then write the append.
   if (lane == 0) {
-    wait_flag_ge(reinterpret_cast<volatile int*>(&a.ctrl[kCtrlPlanned]), G, abort_flag, a.ctrl, 200);
+    // Every launch adds one per CTA, and the grid is the same for every
+    // launch on this cache: this launch is complete at (index + 1) * grid.
+    wait_count_ge(reinterpret_cast<const volatile unsigned long long*>(&a.ctrl[kCtrlPlanned]),
+                  (a.step.launch_index + 1ull) * (unsigned long long)G, abort_flag, a.ctrl, 200);
     fence_acq_rel_gpu();   // acquire: every CTA's reads of the pre-step state happen before our writes
   }
   __syncwarp();
@@ -806,7 +853,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
 
   if (STEP && warp == NCW) {
     step_warp<D, E>(a, nst, prefix, sid, s_nold, s_pos, s_rslot, s_tslot, s_flag, s_rank, misc, healthy,
-                    abort_flag);
+                    abort_flag, K0, K1);
   } else if (STEP || has_range) {
     // ---- this warp's page pipeline: CTA pages c = warp + NCW * j, j = 0 .. njobs-1
     const int njobs = has_range && ncta > warp ? (ncta - warp + NCW - 1) / NCW : 0;
@@ -1080,17 +1127,6 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   // Drain: copies issued but not consumed (only after an abort) must land before exit.
   if (warp < NCW && lane == 0)
     for (int j = consumed; j < issued; ++j) mbar_wait_timed(smem_addr(&myfull[j % spw]), (j / spw) & 1, a.ctrl);
-
-  if constexpr (STEP) {
-    // The last CTA out resets the step's grid counters for the next launch.
-    __syncthreads();
-    if (tid == 0) {
-      if (atomic_add_acq_rel_gpu(&a.ctrl[kCtrlExited], 1) == (int)gridDim.x - 1) {
-        a.ctrl[kCtrlPlanned] = 0;
-        a.ctrl[kCtrlExited] = 0;
-      }
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1238,12 +1274,13 @@ cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t s
 
 cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
                         const void* K, const void* V, const uint8_t* alpha, int alpha_channel, const void* Q, int hq,
-                        float scale, void* out, int out_f32) {
+                        float scale, void* out, int out_f32, unsigned long long launch_index) {
   if (n_seqs == 0) return cudaSuccess;
   AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32);
   a.step.K = (const uint8_t*)K;
   a.step.V = (const uint8_t*)V;
   a.step.asrc = AlphaSrc{alpha, (const uint8_t*)K, alpha_channel, dv.hkv, dv.d, dv.elem_bytes};
+  a.step.launch_index = launch_index;
   a.step.dv = dv;
   return launch_dependent(reinterpret_cast<KernelFn>(plan.fn), dim3(plan.grid), dim3(plan.threads), plan.smem, st,
                           a, plan.tmap);

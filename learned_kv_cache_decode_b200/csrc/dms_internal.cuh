@@ -40,8 +40,8 @@ __device__ __forceinline__ int alpha_at(const AlphaSrc& s, size_t row, int kvh) 
 enum : int {
   kCtrlStatus = 0,   // latched dms_status, 0 = healthy
   kCtrlFree = 1,     // free-stack depth
-  kCtrlPlanned = 2,  // CTAs of a fused decode step done reading the pre-step state
-  kCtrlExited = 3,   // CTAs of a fused decode step that finished
+  kCtrlPlanned = 2,  // words 2-3: uint64 count of fused-step CTAs done reading the pre-step
+                     // state, cumulative over the cache's fused steps (grid per launch)
   kCtrlWords = 8
 };
 
@@ -297,6 +297,28 @@ __device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
 // sequentially consistent fence of __threadfence).
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
+// 64-bit device-scope add with release semantics, no return value.
+__device__ __forceinline__ void red_add_release_gpu_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Spin (one thread) until *counter >= target, sleeping between polls, bounded
+// like wait_flag_ge.
+__device__ __forceinline__ void wait_count_ge(const volatile unsigned long long* counter, unsigned long long target,
+                                              volatile int* abort_flag, int32_t* ctrl, int sleep_ns) {
+  if (*counter >= target) return;
+  const long long t0 = clock64();
+  while (*counter < target) {
+    __nanosleep(sleep_ns);
+    if (*abort_flag) return;
+    if (clock64() - t0 > (1ll << 31)) {
+      latch(ctrl, DMS_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return;
+    }
+  }
+}
+
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -335,7 +357,7 @@ cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int n
 cudaError_t step_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan);
 cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
                         const void* K, const void* V, const uint8_t* alpha, int alpha_channel, const void* Q, int hq,
-                        float scale, void* out, int out_f32);
+                        float scale, void* out, int out_f32, unsigned long long launch_index);
 constexpr int kStepMaxStreams = 1024;   // caches with more streams run the step as two launches
 
 cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,
