@@ -437,7 +437,7 @@ def main():
     t_max_ms, bytes_all = reduce_over_ranks(t_ms, total_bytes, world, dev)
     value = bytes_all / (t_max_ms * 1e-3) / 1e9
 
-    achieved = float(bytes_pl.mean()) / (float(attn_ms.mean()) * 1e-3) / 1e9
+    achieved_iso = float(bytes_pl.mean()) / (float(attn_ms.mean()) * 1e-3) / 1e9
 
     # Burst: `burst_steps` more steps between one event pair, no event between
     # launches, so each launch's set-up overlaps the launch before it
@@ -464,6 +464,24 @@ def main():
     burst_ms = e_b0.elapsed_time(e_b1) / (burst_steps * L)
     b_tot = totals.cpu().numpy()[t_b:t_b + burst_steps]
     achieved_burst = float(b_tot[:, 1].astype(np.float64).mean()) * d * 2 * wl.elem_bytes / (burst_ms * 1e-3) / 1e9
+    # Roofline of the dominant kernel. Fused: the timed region holds the step
+    # launches, back to back as a decode loop issues them, plus one small
+    # dms_stats launch per step, so its average launch duration is this rank's
+    # region time over its step launches (the stats launches count against
+    # it). Separate: the attention launches alone, back to back between one
+    # event pair (the burst). The per-launch event pairs are reported beside
+    # it: an event between two launches makes each start only once the one
+    # before has finished, which removes the overlap of consecutive launches.
+    if fused:
+        launch_ms = t_ms / (args.steps * L)
+        achieved = float(bytes_launch.mean()) / (launch_ms * 1e-3) / 1e9
+        launch_timing = ("timed region (CUDA events at its two ends) over its step launches; "
+                         "isolated: an event pair around every launch, in a second pass over the next steps")
+    else:
+        launch_ms = burst_ms
+        achieved = achieved_burst
+        launch_timing = ("attention launches back to back between one event pair (the burst); "
+                         "isolated: an event pair around every launch, in a second pass over the next steps")
     peak, peak_kind = peaks()
     kernel = {"auto": "mma" if tdt == torch.bfloat16 else "simt"}.get(args.attn_kernel, args.attn_kernel)
 
@@ -575,11 +593,12 @@ def main():
                                                     "dms_decode_step" if fused else "dms_decode_attention"),
                          "kernel": f"dms_decode_step ({kernel}, append fused)" if fused else
                                    f"dms_decode_attention ({kernel})",
-                         "launch_ms_mean": float(attn_ms.mean()), "launch_ms_p10": float(np.percentile(attn_ms, 10)),
-                         "launch_ms_p90": float(np.percentile(attn_ms, 90)),
-                         "bytes_per_launch": float(bytes_pl.mean()),
-                         "launch_timing": "CUDA event pair around every launch, in a second pass over the "
-                                          "next steps; burst: L launches between one event pair",
+                         "bytes_per_launch": float(bytes_launch.mean()) if fused else float(bytes_pl.mean()),
+                         "launch_ms": launch_ms, "launch_timing": launch_timing,
+                         "launch_ms_isolated": float(attn_ms.mean()),
+                         "launch_ms_isolated_p10": float(np.percentile(attn_ms, 10)),
+                         "launch_ms_isolated_p90": float(np.percentile(attn_ms, 90)),
+                         "achieved_isolated": achieved_iso, "frac_isolated": achieved_iso / peak,
                          "launch_ms_burst": burst_ms, "achieved_burst": achieved_burst,
                          "frac_burst": achieved_burst / peak},
             "gpu_launches": launches,

@@ -5,7 +5,10 @@
 // dms_append.cu and dms_attention.cu.
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
+#include <mutex>
 #include <new>
+#include <thread>
 
 #include "dms_internal.cuh"
 
@@ -18,6 +21,12 @@ struct dms_cache {
   dms::AttnPlan step_plan{};   // fused decode step (append + attention in one launch)
   bool has_step = false;       // else dms_decode_step issues the two launches
   uint64_t step_launches = 0;  // fused steps launched since the counters were last cleared
+  // Schedules fused steps leave for the next one (see dms::NextPlan): the tag of
+  // the last fused launch, and the tag the next fused launch may trust (0 once
+  // any other call has changed the cache).
+  dms::NextPlan next{};
+  uint64_t step_tags = 0;
+  uint64_t trust_tag = 0;
   int64_t launches = 0;
   bool poisoned = false;   // a device error was observed by dms_get_status
 };
@@ -25,6 +34,40 @@ struct dms_cache {
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The cache whose kernels were launched last on each stream. Kernels that
+// write a cache are launched only through these calls, so when the record of a
+// stream names another cache, the kernel just before the next launch on that
+// stream (this library's or anyone's) does not write this one. A stream with
+// no record, or one whose record was evicted, counts as this cache's. The
+// per-thread default stream is a different stream in every host thread.
+struct StreamLast {
+  int device;
+  cudaStream_t stream;
+  std::thread::id thread;
+  const dms_cache* cache;
+};
+constexpr int kStreamRecords = 64;
+std::mutex g_last_mu;
+StreamLast g_last[kStreamRecords];
+int g_last_next = 0;
+
+// Records `c` as the last cache launched on `s`; returns true when the
+// previous record of `s` named another cache.
+bool note_launch(const dms_cache* c, int device, cudaStream_t s) {
+  const std::thread::id th = s == cudaStreamPerThread ? std::this_thread::get_id() : std::thread::id();
+  std::lock_guard<std::mutex> lock(g_last_mu);
+  for (StreamLast& e : g_last) {
+    if (e.cache && e.device == device && e.stream == s && e.thread == th) {
+      const bool other = e.cache != c;
+      e.cache = c;
+      return other;
+    }
+  }
+  g_last[g_last_next] = StreamLast{device, s, th, c};
+  g_last_next = (g_last_next + 1) % kStreamRecords;
+  return false;
+}
 
 dms_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DMS_OK : DMS_ERR_CUDA; }
 
@@ -52,6 +95,26 @@ void free_all(dms::Dev& dv) {
 template <typename T>
 cudaError_t alloc(T** p, size_t count) {
   return cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T) + 16);
+}
+
+void free_next(dms::NextPlan& np) {
+  void* ptrs[] = {np.entry, np.hdr, np.list};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  np = dms::NextPlan{};
+}
+
+// Buffers of the schedules a fused step leaves for the next one: one entry per
+// stream, and per tag parity one page list per CTA of the step's grid, long
+// enough for any range (a call holds at most max_pages pages).
+cudaError_t alloc_next(const dms::Dev& dv, int grid, dms::NextPlan* np) {
+  np->cap = (int)std::max<int64_t>(1, ((int64_t)dv.max_pages + grid - 1) / grid);
+  cudaError_t e = alloc(&np->entry, (size_t)dv.S);
+  if (e == cudaSuccess) e = alloc(&np->hdr, (size_t)2 * grid);
+  if (e == cudaSuccess) e = alloc(&np->list, (size_t)2 * grid * np->cap);
+  if (e == cudaSuccess) e = cudaMemset(np->entry, 0, (size_t)dv.S * sizeof(dms::PlanEntry));
+  if (e == cudaSuccess) e = cudaMemset(np->hdr, 0, (size_t)2 * grid * sizeof(int4));
+  return e;
 }
 
 }  // namespace
@@ -114,6 +177,7 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
     h->has_step = dms::step_prepare(dv, c.dtype, c.attn_kernel, h->num_sms, &h->step_plan) == cudaSuccess;
     cudaGetLastError();
   }
+  if (e == cudaSuccess && h->has_step) e = alloc_next(dv, h->step_plan.grid, &h->next);
   const int grid = h->has_step && h->step_plan.grid > h->plan.grid ? h->step_plan.grid : h->plan.grid;
   if (e == cudaSuccess) e = alloc(&dv.part, ((size_t)grid + dv.S) * dms::kMaxGroup * (dv.d + 2));
   if (e == cudaSuccess) e = cudaMemset(dv.kv, 0, (size_t)dv.max_pages * 2 * dms::kPage * dv.d * dv.elem_bytes);
@@ -123,6 +187,7 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     free_all(dv);
+    free_next(h->next);
     delete h;
     cudaGetLastError();
     return e == cudaErrorInvalidValue ? DMS_ERR_INVALID : DMS_ERR_CUDA;
@@ -139,6 +204,7 @@ dms_status dms_cache_destroy(dms_cache* h) {
   cudaSetDevice(h->device);
   cudaError_t e = cudaDeviceSynchronize();
   free_all(h->dv);
+  free_next(h->next);
   if (prev >= 0) cudaSetDevice(prev);
   delete h;
   return from_cuda(e);
@@ -147,6 +213,8 @@ dms_status dms_cache_destroy(dms_cache* h) {
 dms_status dms_cache_reset(dms_cache* h, cudaStream_t stream) {
   if (!h) return DMS_ERR_INVALID;
   if (dms_status s = check_device(h)) return s;
+  h->trust_tag = 0;
+  note_launch(h, h->device, stream);
   cudaError_t e = cudaMemsetAsync(h->dv.page_table, 0xff, (size_t)h->dv.S * h->dv.mps * sizeof(int32_t), stream);
   if (e == cudaSuccess) e = dms::launch_init_state(h->dv, stream);   // clears the step counter too
   h->launches += 1;
@@ -161,6 +229,8 @@ dms_status dms_seq_reset(dms_cache* h, cudaStream_t stream, int32_t seq_id) {
   if (!h || seq_id < 0 || seq_id >= h->cfg.max_seqs) return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
   h->launches += 1;
+  h->trust_tag = 0;
+  note_launch(h, h->device, stream);
   return from_cuda(dms::launch_reset_seq(h->dv, stream, seq_id));
 }
 
@@ -177,6 +247,8 @@ dms_status append_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const 
   if (!aligned16(K) || !aligned16(V)) return DMS_ERR_INVALID;
   int launches = 0;
   cudaError_t e;
+  h->trust_tag = 0;   // the cache changes outside a fused step
+  note_launch(h, h->device, stream);
   if (cu_tokens == nullptr) {
     if (total_tokens != n_seqs) return DMS_ERR_INVALID;
     e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, &launches);
@@ -201,17 +273,24 @@ dms_status step_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const in
   if (!seq_ids || !K || !V || (alpha_channel < 0 && !alpha) || !Q || !out) return DMS_ERR_INVALID;
   if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(out)) return DMS_ERR_INVALID;
   if (!h->has_step) {
+    h->trust_tag = 0;
+    note_launch(h, h->device, stream);
     int launches = 0;
     cudaError_t e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, &launches);
     h->launches += launches;
     if (e != cudaSuccess) return DMS_ERR_CUDA;
     h->launches += 1;
+    note_launch(h, h->device, stream);
     return from_cuda(dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
                                            out_dtype == DMS_F32));
   }
   h->launches += 1;
+  const uint64_t tag = ++h->step_tags;   // consecutive with trust_tag whenever that is set
+  const bool early = note_launch(h, h->device, stream);
   const cudaError_t e = dms::launch_step(h->dv, h->step_plan, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, Q,
-                                         num_q_heads, scale, out, out_dtype == DMS_F32, h->step_launches);
+                                         num_q_heads, scale, out, out_dtype == DMS_F32, h->step_launches, h->next,
+                                         h->trust_tag, tag, early);
+  h->trust_tag = e == cudaSuccess ? tag : 0;
   if (e == cudaSuccess) h->step_launches += 1;
   return from_cuda(e);
 }
@@ -242,6 +321,7 @@ dms_status dms_decode_attention(dms_cache* h, cudaStream_t stream, int32_t n_seq
   if (n_seqs == 0) return DMS_OK;
   if (!seq_ids || !Q || !out || !aligned16(Q) || !aligned16(out)) return DMS_ERR_INVALID;
   h->launches += 1;
+  note_launch(h, h->device, stream);
   return from_cuda(dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
                                          out_dtype == DMS_F32));
 }
@@ -264,6 +344,7 @@ dms_status dms_stats(dms_cache* h, cudaStream_t stream, int32_t* retained, int32
   if (!h) return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
   h->launches += 1;
+  note_launch(h, h->device, stream);
   return from_cuda(dms::launch_stats(h->dv, stream, retained, seen, head_cr, totals));
 }
 
@@ -296,6 +377,7 @@ dms_status dms_gather_kv(dms_cache* h, cudaStream_t stream, int32_t seq_id, int3
   if (rows_cap <= 0) return DMS_OK;
   if (!K_out || !V_out || !aligned16(K_out) || !aligned16(V_out)) return DMS_ERR_INVALID;
   h->launches += 1;
+  note_launch(h, h->device, stream);
   return from_cuda(dms::launch_gather(h->dv, stream, seq_id, kv_head, rows_cap, K_out, V_out));
 }
 

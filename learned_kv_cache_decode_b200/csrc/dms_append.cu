@@ -408,8 +408,13 @@ __global__ void init_state_kernel(Dev dv) {
 // Statistics (one block).
 __global__ void __launch_bounds__(256)
 stats_kernel(Dev dv, int32_t* retained, int32_t* seen, float* head_cr, int64_t* totals) {
+  // Launched behind the previous kernel of the stream (programmatic dependent
+  // launch). The kernel after this one may start at once: what it reads before
+  // its own dependency wait is nothing this kernel writes.
+  grid_dependents_launch();
   __shared__ unsigned long long s_head[kMaxKvHeads][2];
   for (int h = threadIdx.x; h < dv.hkv; h += blockDim.x) s_head[h][0] = s_head[h][1] = 0;
+  grid_dependency_wait();
   __syncthreads();
   for (int st = threadIdx.x; st < dv.S; st += blockDim.x) {
     const int r = dv.n[st], p = dv.pos[st];
@@ -505,8 +510,7 @@ cudaError_t launch_reset_seq(const Dev& dv, cudaStream_t st, int seq) {
 
 cudaError_t launch_stats(const Dev& dv, cudaStream_t st, int32_t* retained, int32_t* seen, float* head_cr,
                          int64_t* totals) {
-  stats_kernel<<<1, 256, 0, st>>>(dv, retained, seen, head_cr, totals);
-  return cudaGetLastError();
+  return launch_dependent(stats_kernel, dim3(1), dim3(256), 0, st, dv, retained, seen, head_cr, totals);
 }
 
 cudaError_t launch_gather(const Dev& dv, cudaStream_t st, int seq, int kvh, int rows_cap, void* Kout,

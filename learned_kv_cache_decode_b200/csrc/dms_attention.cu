@@ -43,6 +43,7 @@ namespace dms {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kRslotUnknown = -2;   // leaving slot not known until the window ring is read
 
 // A decode step fused into the attention launch: the new token of every call
 // stream and the cache the append writes.
@@ -52,6 +53,10 @@ struct StepArgs {
   AlphaSrc asrc;          // eviction decisions of the new tokens
   unsigned long long launch_index;   // fused steps launched on this cache before this one
   Dev dv;                 // the cache, writable
+  NextPlan next;          // schedule left by the previous fused step, and the one this step leaves
+  unsigned long long trust;   // tag of the schedule to read (0: none, plan from the cache state)
+  unsigned long long wtag;    // tag of the schedule this launch writes (trust + 1 when trust != 0)
+  int pre;                    // the kernel before this one in the stream does not write this cache
 };
 
 struct AttnArgs {
@@ -585,9 +590,10 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
     const bool fits = total <= fc;
     int rank = incl - cnt;
     for (int i = b0; i < e0; ++i) {
+      s_rank[i] = fits ? rank : 0;   // pages popped by the streams before i (a popping stream's rank)
       if (!(s_flag[i] & 1)) continue;
       if (fits) {
-        s_rank[i] = rank++;
+        ++rank;
       } else {
         s_tslot[i] = -1;   // pool exhausted: this stream is left unchanged
         s_flag[i] |= 16;
@@ -643,6 +649,57 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
     }
   }
 
+  // This CTA's page list for the next step on the same streams. After this
+  // step, stream i holds its old pages plus the one it popped, so its pages
+  // start at prefix[i] + s_rank[i] in the call's concatenated order, and the
+  // next step cuts P + pops pages into the same kind of ranges. Existing pages
+  // come from the page table (this step writes only entries past them), a
+  // popped one from the free stack (never written by a step). Nothing reads
+  // this buffer during this launch: it is the one of the other tag parity.
+  // Eight loads per lane are in flight at a time.
+  if (a.step.next.entry != nullptr && misc[13] >= 0) {
+    const long long P2 = (long long)prefix[nst] + misc[13];
+    const long long Ge = P2 < G ? P2 : G;
+    const long long c0 = blockIdx.x < Ge ? blockIdx.x * P2 / Ge : 0;
+    const long long c1 = blockIdx.x < Ge ? (blockIdx.x + 1) * P2 / Ge : 0;
+    if (c1 - c0 <= a.step.next.cap) {
+      const size_t cell = (size_t)(a.step.wtag & 1ull) * G + blockIdx.x;
+      int32_t* lst = a.step.next.list + cell * a.step.next.cap;
+      const int fc = misc[12];
+      for (long long base = c0; base < c1; base += 32 * 8) {
+        int v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const long long kk = base + lane + 32 * u;
+          v[u] = 0;
+          if (kk < c1) {
+            int lo = 0, hi = nst;   // largest i with prefix[i] + s_rank[i] <= kk
+            while (hi - lo > 1) {
+              const int mid = (lo + hi) >> 1;
+              if (prefix[mid] + s_rank[mid] <= kk) lo = mid; else hi = mid;
+            }
+            const int p = (int)(kk - prefix[lo] - s_rank[lo]);
+            v[u] = p < prefix[lo + 1] - prefix[lo] ? __ldg(dv.page_table + (size_t)sid[lo] * dv.mps + p)
+                                                   : __ldg(dv.free_list + (fc - 1 - s_rank[lo]));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const long long kk = base + lane + 32 * u;
+          if (kk < c1) lst[kk - c0] = v[u];
+        }
+      }
+      __syncwarp();
+      if (lane == 0)
+        a.step.next.hdr[cell] = make_int4((int)(uint32_t)a.step.wtag, (int)(uint32_t)(a.step.wtag >> 32), nst, (int)P2);
+    }
+  }
+  // The window-ring entry the next step reads for this CTA's first stream
+  // (residue s + 1, which this step does not write when w > 1), requested now.
+  int rn_first = 0;
+  if (a.step.next.entry != nullptr && lane == 0 && blockIdx.x < nst && dv.w > 1 && s_tslot[blockIdx.x] >= 0)
+    rn_first = dv.ring[(size_t)sid[blockIdx.x] * dv.w + ((s_pos[blockIdx.x] + 1) % dv.w)];
+
   // Wait until every CTA has read the pre-step state, then write the append.
   if (lane == 0) {
     // Every launch adds one per CTA, and the grid is the same for every
@@ -674,20 +731,50 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
       continue;
     }
     if (lane == 0) {
+      const int nnew = s_rslot[i] < 0 ? s_nold[i] + 1 : s_nold[i];
+      const int rent = (ts << 1) | ((f >> 1) & 1);
       if (f & 1) {
         dv.page_table[(size_t)st * dv.mps + lp] = page;
         dv.n_pages[st] = lp + 1;
       }
-      if (s_rslot[i] < 0) dv.n[st] = s_nold[i] + 1;
-      dv.ring[(size_t)st * dv.w + (s % dv.w)] = (ts << 1) | ((f >> 1) & 1);
+      if (s_rslot[i] < 0) dv.n[st] = nnew;
+      dv.ring[(size_t)st * dv.w + (s % dv.w)] = rent;
       dv.pos[st] = s + 1;
       dv.slot_pos[(size_t)page * kPage + ts % kPage] = s;
+      if (a.step.next.entry != nullptr) {
+        // The schedule entry of call stream i for the next step. Its window-ring
+        // entry is the one at residue s + 1: the one just written when w = 1,
+        // else one this step leaves alone.
+        const int rnext = dv.w == 1 ? rent
+                          : (i == (int)blockIdx.x ? rn_first : dv.ring[(size_t)st * dv.w + ((s + 1) % dv.w)]);
+        PlanEntry* e = a.step.next.entry + i;
+        *reinterpret_cast<int4*>(e) = make_int4(nnew, s + 1, rnext, st / a.hkv);
+        e->tag = a.step.wtag;
+      }
     }
     for (int v = lane; v < 2 * vec; v += 32) {
       const int which = v / vec, c = v % vec;
       const uint4 x = __ldg(reinterpret_cast<const uint4*>((which ? a.step.V : a.step.K) + (size_t)i * row_bytes) + c);
       reinterpret_cast<uint4*>(dv.kv + ((size_t)page * 2 * kPage + (size_t)which * kPage + ts % kPage) * row_bytes)[c] = x;
     }
+  }
+}
+
+// One page (16 K rows, then 16 V rows) into a warp's stage j % spw, completing
+// on that stage's mbarrier. Called by one lane.
+template <int D, bool MMA, typename E>
+__device__ __forceinline__ void issue_page(uint64_t* myfull, uint8_t* mystage, int spw, int j, int pg,
+                                           const CUtensorMap* tmap, const uint8_t* kv) {
+  constexpr int kStage = 2 * kPage * D * (int)sizeof(E);
+  const int s = j % spw;
+  const uint32_t bar = smem_addr(&myfull[s]);
+  const uint32_t dst = smem_addr(mystage + (size_t)s * kStage);
+  mbar_arrive_expect_tx(bar, kStage);
+  if constexpr (MMA) {
+#pragma unroll
+    for (int box = 0; box < D / 64; ++box) tma_load_3d(dst + box * 4096, tmap, bar, box * 64, 0, pg);
+  } else {
+    bulk_load(dst, kv + (size_t)pg * kStage, kStage, bar);
   }
 }
 
@@ -775,41 +862,189 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   volatile int* abort_flag = misc;
 
   if (tid == 0) {
+    if constexpr (MMA) prefetch_tensormap(&tmap);
     misc[0] = 0;
     misc[14] = -1;
     misc[15] = 0;
     for (int s = 0; s < NCW * spw; ++s) mbar_init(smem_addr(&full[s]), 1);
     fence_mbar_init();
   }
+  // Call streams [b0, e0) of this thread in the plan.
+  const int per = (nst + kThreads - 1) / kThreads;
+  const int b0 = min(tid * per, nst), e0 = min(b0 + per, nst);
+
+  // STEP: the schedule the previous fused step left (counts, positions and
+  // leaving slots after it, this CTA's page ids), trusted when the host says
+  // no other call has changed the cache since.
+  const unsigned long long trust = STEP ? a.step.trust : 0ull;
+  const int tbuf = (int)(trust & 1ull);
+  int4 thdr = make_int4(0, 0, 0, 0);   // header of this CTA's page list in it
+  int spec_pg = 0;                     // consumer lanes: page id of the warp's job `lane` in it
+  auto load_schedule_head = [&]() {
+    const size_t cell = (size_t)tbuf * gridDim.x + blockIdx.x;
+    thdr = ld_early4(a.step.next.hdr + cell);
+    if (warp < NCW && warp + NCW * lane < a.step.next.cap)
+      spec_pg = ld_early(a.step.next.list + cell * a.step.next.cap + warp + NCW * lane);
+  };
+  // This CTA's page ids come from the schedule when every stream of the call
+  // matched it (same streams in the same order, hence the same counts and the
+  // same partition) and its page list was written for exactly this call.
+  auto list_matches = [&](long long P_, int ncta_, bool any_miss_) -> bool {
+    const bool head = (unsigned long long)(uint32_t)thdr.x + ((unsigned long long)(uint32_t)thdr.y << 32) == trust &&
+                      thdr.z == nst;
+    thdr = make_int4(0, 0, 0, head ? thdr.w : -1);   // only the page count is needed from here on
+    return STEP && trust != 0 && !any_miss_ && head && thdr.w == (int)P_ && ncta_ <= a.step.next.cap;
+  };
+
+  // STEP, early start. When the host knows that the kernel just before this
+  // one in the stream does not write this cache, everything the schedule
+  // describes (and the cache pages themselves) is final before the dependency
+  // wait; only the call's own inputs (seq ids, alpha, queries, new rows) may
+  // still be in the making. The plan and the first page copies then go ahead
+  // of the wait on the guess that the call has the streams of the step that
+  // wrote the schedule, which the seq ids confirm after it. This overlaps the
+  // start of this launch with the end of the previous one.
+  bool pre_ok = false;     // CTA-uniform: planned and copies issued before the wait
+  bool any_miss = true;    // some stream of the call did not match the schedule
+  if (STEP && trust != 0 && a.step.pre != 0) {
+    load_schedule_head();
+    const int status = tid == 0 ? read_status(a.ctrl) : 0;
+    const int free_depth = tid == 0 ? *reinterpret_cast<const volatile int32_t*>(&a.ctrl[kCtrlFree]) : 0;
+    bool miss = false;
+    int local = 0;
+    for (int i = b0; i < e0; ++i) {
+      const int4 en = ld_early4(reinterpret_cast<const int4*>(a.step.next.entry + i));
+      const unsigned long long etag = ld_early_u64(&a.step.next.entry[i].tag);
+      const bool ok = etag == trust && en.w >= 0 && en.w < a.max_seqs;
+      const int nn = ok ? en.x : 0;
+      s_nold[i] = nn;
+      s_pos[i] = en.y;
+      s_flag[i] = 0;
+      s_rslot[i] = ok && en.y >= a.step.dv.w && (en.z & 1) ? (en.z >> 1) : -1;
+      sid[i] = ok ? en.w * a.hkv + i % a.hkv : 0;
+      prefix[i + 1] = (nn + kPage - 1) / kPage;
+      local += prefix[i + 1];
+      miss |= !ok;
+    }
+    int total;
+    int run = block_exclusive_scan(local, misc + 3, &total);
+    for (int i = b0; i < e0; ++i) {
+      run += prefix[i + 1];
+      prefix[i + 1] = run;
+    }
+    if (tid == 0) {
+      prefix[0] = 0;
+      misc[1] = (status == 0);
+      misc[12] = free_depth;
+    }
+    any_miss = __syncthreads_or(miss) != 0;
+    const long long P0 = prefix[nst];
+    const long long G0 = P0 < gridDim.x ? P0 : gridDim.x;
+    const int k0 = blockIdx.x < G0 ? (int)(blockIdx.x * P0 / G0) : 0;
+    const int k1 = blockIdx.x < G0 ? (int)((blockIdx.x + 1) * P0 / G0) : 0;
+    pre_ok = misc[1] != 0 && list_matches(P0, k1 - k0, any_miss);
+    if (pre_ok && warp < NCW) {
+      const int nj = k1 - k0 > warp ? (k1 - k0 - warp + NCW - 1) / NCW : 0;
+      for (int j = 0; j < spw && j < nj; ++j) {
+        int pg = __shfl_sync(0xffffffffu, spec_pg, j);
+        if (lane == 0) {
+          if (pg < 0 || pg >= a.max_pages) {
+            latch(a.ctrl, DMS_ERR_INVALID);
+            pg = 0;
+          }
+          issue_page<D, MMA, E>(full + warp * spw, smem + lay.stages + (size_t)warp * spw * kStage, spw, j, pg,
+                                &tmap, a.kv);
+        }
+      }
+    }
+  }
+
   // Launched early behind the previous kernel of the stream (programmatic
   // dependent launch): everything above overlaps it; nothing it writes is
   // read before this point.
   grid_dependency_wait();
 
+  if (pre_ok) {
+    // The call's seq ids against the guess, and the alpha of its new tokens.
+    bool bad = false;
+    for (int i = b0; i < e0; ++i) {
+      const int seq = a.seq_ids[i / a.hkv];
+      const int al = alpha_at(a.step.asrc, (size_t)(i / a.hkv), i % a.hkv);
+      bad |= seq != sid[i] / a.hkv;
+      s_flag[i] = al != 0 ? 2 : 0;
+    }
+    if (__syncthreads_or(bad)) {
+      // Another call: let the guessed copies land, then take every stage
+      // barrier of the warp exactly two phases on with plain arrivals (one
+      // after a landed copy, two on an unused stage), so that each is back at
+      // a phase of parity 0 as the pipeline expects; then plan from the seq ids.
+      if (warp < NCW && lane == 0) {
+        const long long P0 = prefix[nst];
+        const long long G0 = P0 < gridDim.x ? P0 : gridDim.x;
+        const int k0 = blockIdx.x < G0 ? (int)(blockIdx.x * P0 / G0) : 0;
+        const int k1 = blockIdx.x < G0 ? (int)((blockIdx.x + 1) * P0 / G0) : 0;
+        const int nj = min(spw, k1 - k0 > warp ? (k1 - k0 - warp + NCW - 1) / NCW : 0);
+        for (int j = 0; j < spw; ++j) {
+          const uint32_t bar = smem_addr(&full[warp * spw + j]);
+          if (j < nj) {
+            mbar_wait_timed(bar, 0, a.ctrl);
+          } else {
+            mbar_arrive(bar);
+          }
+          mbar_arrive(bar);
+        }
+      }
+      __syncthreads();   // prefix is read above before the plan below rewrites it
+      pre_ok = false;
+    }
+  }
+
   // ---- plan: retained pages per stream of the call (prefix) and stream ids,
   // in smem. The status word is read in the same round trip as the seq ids.
-  {
+  // STEP: so are the schedule entries (a stream whose entry does not match
+  // falls back to the cache state) and this CTA's page ids from it.
+  if (!pre_ok) {
+    if (STEP && trust != 0) load_schedule_head();
+    // Both control words are kept in registers until the loop's loads are out:
+    // a shared-memory store of a loaded value here would hold them back one
+    // round trip.
     const int status = tid == 0 ? read_status(a.ctrl) : 0;
-    if (STEP && tid == 0) misc[12] = *reinterpret_cast<const volatile int32_t*>(&a.ctrl[kCtrlFree]);
-    const int per = (nst + kThreads - 1) / kThreads;
-    const int b0 = min(tid * per, nst), e0 = min(b0 + per, nst);
+    const int free_depth = (STEP && tid == 0) ? *reinterpret_cast<const volatile int32_t*>(&a.ctrl[kCtrlFree]) : 0;
+    bool miss = !STEP || trust == 0;
     int local = 0;
     for (int i = b0; i < e0; ++i) {
       const int seq = a.seq_ids[i / a.hkv];
       const int al = STEP ? alpha_at(a.step.asrc, (size_t)(i / a.hkv), i % a.hkv) : 0;   // same round trip as the seq id
+      int4 en = make_int4(0, 0, 0, -1);
+      unsigned long long etag = 0;
+      if (STEP && trust != 0) {
+        en = ld_early4(reinterpret_cast<const int4*>(a.step.next.entry + i));
+        etag = ld_early_u64(&a.step.next.entry[i].tag);
+      }
       int pages = 0, st = 0;
       if (seq < 0 || seq >= a.max_seqs) {
-        if constexpr (STEP) s_flag[i] = 4;   // latched once every CTA has read the status
-        else latch(a.ctrl, DMS_ERR_BAD_SEQ);
+        if constexpr (STEP) {
+          s_flag[i] = 4;   // latched once every CTA has read the status
+          s_rslot[i] = -1;
+        } else {
+          latch(a.ctrl, DMS_ERR_BAD_SEQ);
+        }
+        miss = true;
       } else {
         st = seq * a.hkv + i % a.hkv;
-        const int nn = a.n[st];
+        const bool hit = STEP && trust != 0 && etag == trust && en.w == seq;
+        const int nn = hit ? en.x : a.n[st];
         pages = (nn + kPage - 1) / kPage;
         if constexpr (STEP) {
+          const int ps = hit ? en.y : a.step.dv.pos[st];
           s_nold[i] = nn;
-          s_pos[i] = a.step.dv.pos[st];
+          s_pos[i] = ps;
           s_flag[i] = al != 0 ? 2 : 0;
+          // The token at ps - w leaves now if it was marked; unknown until the
+          // window ring is read when the schedule had no entry.
+          s_rslot[i] = hit ? ((ps >= a.step.dv.w && (en.z & 1)) ? (en.z >> 1) : -1) : kRslotUnknown;
         }
+        miss |= !hit;
       }
       sid[i] = st;
       prefix[i + 1] = pages;
@@ -824,9 +1059,10 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     if (tid == 0) {
       prefix[0] = 0;
       misc[1] = (status == 0);
+      if (STEP) misc[12] = free_depth;
     }
+    any_miss = __syncthreads_or(miss) != 0;
   }
-  __syncthreads();
   grid_dependents_launch();   // the next kernel may queue up behind this one
   const bool healthy = misc[1] != 0;
   if constexpr (!STEP) {
@@ -848,6 +1084,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   const int K0 = has_range ? (int)(blockIdx.x * P / Geff) : 0;
   const int K1 = has_range ? (int)((blockIdx.x + 1) * P / Geff) : 0;
   const int ncta = K1 - K0;
+  const bool list_ok = list_matches(P, ncta, any_miss);
   int consumed = 0, issued = 0;
   uint64_t* myfull = full + (warp < NCW ? warp : 0) * spw;
 
@@ -858,16 +1095,21 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     // ---- this warp's page pipeline: CTA pages c = warp + NCW * j, j = 0 .. njobs-1
     const int njobs = has_range && ncta > warp ? (ncta - warp + NCW - 1) / NCW : 0;
     uint8_t* mystage = smem + lay.stages + (size_t)warp * spw * kStage;
-    auto lookup = [&](int j) -> int {   // physical page of the warp's j-th page
-      if (j >= njobs) return 0;
-      const int kk = K0 + warp + NCW * j;
-      const int i = stream_of(prefix, nst, kk);
-      int pg = __ldg(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i]));
+    const int32_t* tlist = STEP ? a.step.next.list + ((size_t)tbuf * gridDim.x + blockIdx.x) * a.step.next.cap
+                                : nullptr;
+    auto checked = [&](int pg) -> int {
       if (pg < 0 || pg >= a.max_pages) {
         latch(a.ctrl, DMS_ERR_INVALID);
         pg = 0;
       }
       return pg;
+    };
+    auto lookup = [&](int j) -> int {   // physical page of the warp's j-th page
+      if (j >= njobs) return 0;
+      if (STEP && list_ok) return checked(__ldg(tlist + warp + NCW * j));
+      const int kk = K0 + warp + NCW * j;
+      const int i = stream_of(prefix, nst, kk);
+      return checked(__ldg(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i])));
     };
     using State = typename std::conditional<MMA, MmaState<D>, SimtState<D>>::type;
     using Query = typename std::conditional<MMA, MmaQuery<D>, SimtQuery<D>>::type;
@@ -899,13 +1141,14 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
 #pragma unroll
       for (int q = 0; q < kRingPer; ++q) {
         const int il = tid + q * kMergeThreads;
-        ring_v[q] = (il < nst && !(s_flag[il] & 4))
+        ring_v[q] = (il < nst && s_rslot[il] == kRslotUnknown)
                         ? ld_early(a.step.dv.ring + (size_t)sid[il] * a.step.dv.w + (s_pos[il] % a.step.dv.w))
                         : 0;
       }
     }
-    int jb = 0;                                     // page ids of jobs [jb, jb+32) in pid_cur,
-    int pid_cur = lookup(lane), pid_nxt = lookup(32 + lane);   // [jb+32, jb+64) in pid_nxt
+    int jb = 0;   // page ids of jobs [jb, jb+32) in pid_cur, [jb+32, jb+64) in pid_nxt
+    int pid_cur = (STEP && list_ok) ? (lane < njobs ? checked(spec_pg) : 0) : lookup(lane);
+    int pid_nxt = lookup(32 + lane);
     auto issue = [&](int j) {   // warp-uniform; j = issued
       if (j - jb >= 32) {
         pid_cur = pid_nxt;
@@ -914,31 +1157,20 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       }
       const int r = j - jb;
       const int pg = __shfl_sync(0xffffffffu, r < 32 ? pid_cur : pid_nxt, r & 31);
-      if (lane == 0) {
-        const int s = j % spw;
-        const uint32_t bar = smem_addr(&myfull[s]);
-        const uint32_t dst = smem_addr(mystage + (size_t)s * kStage);
-        mbar_arrive_expect_tx(bar, kStage);
-        if constexpr (MMA) {
-#pragma unroll
-          for (int box = 0; box < D / 64; ++box) tma_load_3d(dst + box * 4096, &tmap, bar, box * 64, 0, pg);
-        } else {
-          bulk_load(dst, a.kv + (size_t)pg * kStage, kStage, bar);
-        }
-      }
+      if (lane == 0) issue_page<D, MMA, E>(myfull, mystage, spw, j, pg, &tmap, a.kv);
       issued = j + 1;
     };
-    for (int j = 0; j < spw && j < njobs; ++j) issue(j);
+    if (pre_ok) issued = min(spw, njobs);   // the first copies went out before the dependency wait
+    else
+      for (int j = 0; j < spw && j < njobs; ++j) issue(j);
     if constexpr (STEP) {
       // The logical slot of the token leaving at this step (-1: none), for the
       // consumers' masks and the step warp's decisions.
 #pragma unroll
       for (int q = 0; q < kRingPer; ++q) {
         const int il = tid + q * kMergeThreads;
-        if (il < nst && !(s_flag[il] & 4))
+        if (il < nst && s_rslot[il] == kRslotUnknown)
           s_rslot[il] = (s_pos[il] >= a.step.dv.w && (ring_v[q] & 1)) ? (ring_v[q] >> 1) : -1;
-        else if (il < nst)
-          s_rslot[il] = -1;
       }
       named_barrier_arrive(2, kThreads);   // hand them to the step warp (which syncs on barrier 2)
     }
@@ -1274,14 +1506,23 @@ cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t s
 
 cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
                         const void* K, const void* V, const uint8_t* alpha, int alpha_channel, const void* Q, int hq,
-                        float scale, void* out, int out_f32, unsigned long long launch_index) {
+                        float scale, void* out, int out_f32, unsigned long long launch_index,
+                        const NextPlan& next, unsigned long long trust_tag, unsigned long long write_tag,
+                        bool early) {
   if (n_seqs == 0) return cudaSuccess;
+  // A schedule is read from the buffer of its tag's parity and written to the
+  // other one, so the two tags must be consecutive.
+  if (write_tag == 0 || (trust_tag != 0 && trust_tag + 1 != write_tag)) return cudaErrorInvalidValue;
   AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32);
   a.step.K = (const uint8_t*)K;
   a.step.V = (const uint8_t*)V;
   a.step.asrc = AlphaSrc{alpha, (const uint8_t*)K, alpha_channel, dv.hkv, dv.d, dv.elem_bytes};
   a.step.launch_index = launch_index;
   a.step.dv = dv;
+  a.step.next = next;
+  a.step.trust = next.entry ? trust_tag : 0ull;
+  a.step.wtag = write_tag;
+  a.step.pre = early ? 1 : 0;
   return launch_dependent(reinterpret_cast<KernelFn>(plan.fn), dim3(plan.grid), dim3(plan.threads), plan.smem, st,
                           a, plan.tmap);
 }

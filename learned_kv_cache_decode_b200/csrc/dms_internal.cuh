@@ -185,6 +185,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Bring a tensor map into the TMA unit's descriptor cache ahead of its first
+// copy (the map is a kernel parameter, readable before any dependency wait).
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 // Untiled bulk copy global -> shared (size and both addresses 16-B aligned).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
@@ -252,6 +258,19 @@ __device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
 __device__ __forceinline__ int ld_early(const int32_t* p) {
   int v;
   asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int4 ld_early4(const int4* p) {   // p 16-byte aligned
+  int4 v;
+  asm volatile("ld.global.cg.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned long long ld_early_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.global.cg.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 
@@ -355,9 +374,43 @@ struct AttnPlan {
 cudaError_t attention_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan);
 // The fused decode step (append + attention in one launch); see dms_decode_step.
 cudaError_t step_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, AttnPlan* plan);
+
+// The schedule a fused decode step leaves for the next one on the same cache.
+// Decode calls the step again and again with the same sequences; the step that
+// has just resolved every stream's slots already knows the next step's
+// retained counts, positions, leaving slots and page partition, so it writes
+// them down and the next step starts its page copies after one round trip
+// instead of three (seq ids, then counts, then page ids and window-ring
+// entries). The host tags every fused launch (`tag`, never reused) and tells
+// the next one which tag to trust: that of the fused step immediately before
+// it, or none when another call has changed the cache in between.
+//
+// Entry i describes call stream i after the step that wrote it.
+struct __align__(16) PlanEntry {
+  int32_t n, pos;       // retained tokens, tokens seen
+  int32_t ring;         // window-ring entry of the token that leaves at the next step
+  int32_t seq;          // sequence id of call stream i (stream = seq * hkv + i % hkv)
+  unsigned long long tag;
+  int32_t pad[2];
+};
+// Page list of CTA c for the next step: the physical page ids of its range, in
+// range order, with a header {tag lo, tag hi, call streams, total pages}.
+// Double-buffered by tag parity: a step reads the buffer of the tag it trusts
+// while it writes the other one.
+struct NextPlan {
+  PlanEntry* entry;   // [S]
+  int4* hdr;          // [2][grid]
+  int32_t* list;      // [2][grid][cap]
+  int cap;            // page ids per CTA: enough for any range of any call (max_pages / grid, rounded up)
+};
+// `early`: the host knows that the kernel just before this launch in its stream
+// does not write this cache, so the step may plan from the schedule and start
+// its first page copies before its dependency wait (checked after it).
 cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
                         const void* K, const void* V, const uint8_t* alpha, int alpha_channel, const void* Q, int hq,
-                        float scale, void* out, int out_f32, unsigned long long launch_index);
+                        float scale, void* out, int out_f32, unsigned long long launch_index,
+                        const NextPlan& next, unsigned long long trust_tag, unsigned long long write_tag,
+                        bool early);
 constexpr int kStepMaxStreams = 1024;   // caches with more streams run the step as two launches
 
 cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,

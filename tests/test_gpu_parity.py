@@ -306,6 +306,59 @@ def test_fused_step_bad_seq_latches():
         run.close()
 
 
+SCHEDULE_CASES = [
+    wl("schedule-bf16-g7-d128", 6, 14, 2, 128, "bf16", 8, (1, 500), 0, 0.6, 34),
+    wl("schedule-bf16-g4-d64-w1", 6, 8, 2, 64, "bf16", 1, (10, 300), 0, 0.5, 35),
+    wl("schedule-f32-g4-d64", 5, 8, 2, 64, "f32", 24, (1, 400), 0, 0.5, 36),
+]
+
+
+@pytest.mark.parametrize("case", SCHEDULE_CASES, ids=[c.name for c in SCHEDULE_CASES])
+@pytest.mark.parametrize("caches", [1, 2], ids=["one_cache", "two_caches_interleaved"])
+def test_fused_step_schedule_follows_every_change(case, caches):
+    """A fused step leaves the next one its schedule (counts, positions, leaving slots,
+    page lists). Drive it through every way that schedule can stop matching: the same
+    streams again, a permuted order, a prefix subset, a superset, a two-launch step in
+    between, a sequence restart, and back. Metadata bit for bit and every output against
+    the oracle, at every step.
+
+    With two caches stepped in turn on one stream, the kernel before each fused step is
+    the other cache's, so the step plans from the schedule and issues its first copies
+    before its dependency wait, and checks the guess against the seq ids after it (a
+    changed stream list takes the fallback: drain, reset the stage barriers, re-plan)."""
+    B = case.batch
+    perm = [3, 1, 0, 4, 2] + list(range(5, B))
+    plan = ([("fused", list(range(B)))] * 4 + [("fused", perm)] * 2 + [("fused", perm[:3])] +
+            [("fused", perm)] * 2 + [("two", list(range(B)))] + [("fused", list(range(B)))] * 3 +
+            [("reset", 2)] + [("fused", list(range(B)))] * 3 + [("fused", list(range(B))[::-1])] * 2)
+    runs = [Run(case, steps=len(plan)) for _ in range(caches)]
+    tol = dict(max_abs=1e-4, mean_abs=1e-5) if case.dtype == "f32" else {}
+    try:
+        for run in runs:
+            run.prefill(chunk=97)
+            run.check_metadata()
+        for step, (kind, arg) in enumerate(plan):
+            for run in runs:
+                if kind == "reset":
+                    run.cache.reset_seq(arg)
+                    assert run.sim.reset_seq(arg) == 0
+                    run.seen[arg] = 0
+                    run._blk.pop(arg, None)
+                    run.prefill(chunk=97, seqs=[arg])
+                    continue
+                out, Q = run.decode_step(step, seqs=arg, fused=kind == "fused")
+                torch.cuda.synchronize()
+                for j, b in enumerate(arg):
+                    compare(out[j], run.oracle_out(b, Q[j]), **tol)
+            for run in runs:
+                run.check_metadata()
+        for run in runs:
+            assert run.cache.status() == _native.DMS_OK
+    finally:
+        for run in runs:
+            run.close()
+
+
 # ---------------------------------------------------------------------------
 # alpha read from a designated key channel (dms_append_keyed, dms_decode_step_keyed)
 
