@@ -169,7 +169,20 @@ dms_status dms_decode_attention(dms_cache* cache, cudaStream_t stream, int32_t n
  * from K and V; the append's writes go to rows that no part of the launch
  * attends. A cache with more than 1024 streams (max_seqs * num_kv_heads), or
  * whose configuration leaves no shared memory for the step's per-stream
- * state, issues the two launches instead.
+ * state, issues the two launches instead; so does a call on a stream that is
+ * being captured into a CUDA graph (the fused launch carries host sequence
+ * numbers and cannot be replayed).
+ * Each fused step leaves the next one on the same cache a schedule: every
+ * call stream's count, position and leaving slot after it, and the page ids
+ * of every CTA's range. The next fused step uses it when no other call has
+ * changed the cache in between (it checks the entries against its seq ids
+ * and falls back stream by stream), which saves it two dependent memory
+ * round trips. When, in addition, the kernel just before it in the stream is
+ * not one of this cache's, it plans and starts its first page copies before
+ * that kernel has finished (programmatic dependent launch), on the guess that
+ * its seq ids are those of the step that left the schedule; the guess is
+ * checked once the previous kernel is done. Calls on one cache must run in
+ * the order they are made: on one stream, or on streams ordered by events.
  *   n_seqs, seq_ids      as dms_append (one token per sequence)
  *   K, V                 device [n_seqs, num_kv_heads, head_dim] of the cache dtype, 16-B aligned
  *   alpha                device uint8 [n_seqs, num_kv_heads]

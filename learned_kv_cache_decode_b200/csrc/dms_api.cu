@@ -272,7 +272,16 @@ dms_status step_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const in
   if (n_seqs == 0) return DMS_OK;
   if (!seq_ids || !K || !V || (alpha_channel < 0 && !alpha) || !Q || !out) return DMS_ERR_INVALID;
   if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(out)) return DMS_ERR_INVALID;
-  if (!h->has_step) {
+  // A fused launch carries host sequence numbers (the launch index its
+  // grid-wide counter is checked against, the schedule tags), so a graph
+  // replay of it would be wrong: under stream capture the step is issued as
+  // the two launches, which replay as they were captured.
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess) {
+    cudaGetLastError();
+    return DMS_ERR_CUDA;
+  }
+  if (!h->has_step || capture != cudaStreamCaptureStatusNone) {
     h->trust_tag = 0;
     note_launch(h, h->device, stream);
     int launches = 0;

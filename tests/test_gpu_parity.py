@@ -11,7 +11,7 @@ import torch
 
 from learned_kv_cache_decode_b200 import workloads as W
 from learned_kv_cache_decode_b200 import _native
-from harness import Run, compare
+from harness import Run, compare, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -357,6 +357,48 @@ def test_fused_step_schedule_follows_every_change(case, caches):
     finally:
         for run in runs:
             run.close()
+
+
+def test_decode_step_captured_in_a_cuda_graph_replays_step_after_step():
+    """dms_decode_step captured into a CUDA graph (issued as dms_append +
+    dms_decode_attention under capture), replayed once per decode step with the
+    step's inputs copied into the captured buffers: metadata bit for bit and every
+    output against the oracle."""
+    case = wl("graph-bf16-g7-d128", 3, 21, 3, 128, "bf16", 16, (40, 600), 6, 0.6, 37)
+    run = Run(case)
+    try:
+        run.prefill(chunk=97)
+        seqs = list(range(case.batch))
+        K, V, A, Q = run.decode_inputs(0, seqs)
+        ids = torch.tensor(seqs, dtype=torch.int32, device="cuda")
+        dK, dV, dQ = to_device(K, case), to_device(V, case), to_device(Q, case)
+        dA = torch.from_numpy(A).cuda()
+        out = torch.empty_like(dQ)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run.cache.decode_step(ids, dK, dV, dA, dQ, scale=run.scale, out=out)
+        # capture only records the launches: the cache is unchanged so far
+        run.check_metadata()
+        for step in range(case.decode_steps):
+            K, V, A, Q = run.decode_inputs(step, seqs)
+            dK.copy_(to_device(K, case))
+            dV.copy_(to_device(V, case))
+            dA.copy_(torch.from_numpy(A))
+            dQ.copy_(to_device(Q, case))
+            g.replay()
+            torch.cuda.synchronize()
+            rc, _ = run.sim.append(seqs, [1] * len(seqs), A)
+            assert rc == 0
+            for b in seqs:
+                run.seen[b] += 1
+            for b in seqs:
+                compare(out[b], run.oracle_out(b, Q[b]))
+            run.check_metadata()
+        assert run.cache.status() == _native.DMS_OK
+        del g
+    finally:
+        run.close()
 
 
 # ---------------------------------------------------------------------------
