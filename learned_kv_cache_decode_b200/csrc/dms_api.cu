@@ -110,10 +110,10 @@ void free_next(dms::NextPlan& np) {
 cudaError_t alloc_next(const dms::Dev& dv, int grid, dms::NextPlan* np) {
   np->cap = (int)std::max<int64_t>(1, ((int64_t)dv.max_pages + grid - 1) / grid);
   cudaError_t e = alloc(&np->entry, (size_t)dv.S);
-  if (e == cudaSuccess) e = alloc(&np->hdr, (size_t)2 * grid);
+  if (e == cudaSuccess) e = alloc(&np->hdr, (size_t)2 * grid * 2);
   if (e == cudaSuccess) e = alloc(&np->list, (size_t)2 * grid * np->cap);
   if (e == cudaSuccess) e = cudaMemset(np->entry, 0, (size_t)dv.S * sizeof(dms::PlanEntry));
-  if (e == cudaSuccess) e = cudaMemset(np->hdr, 0, (size_t)2 * grid * sizeof(int4));
+  if (e == cudaSuccess) e = cudaMemset(np->hdr, 0, (size_t)2 * grid * 2 * sizeof(int4));
   return e;
 }
 

@@ -690,8 +690,10 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
         }
       }
       __syncwarp();
-      if (lane == 0)
-        a.step.next.hdr[cell] = make_int4((int)(uint32_t)a.step.wtag, (int)(uint32_t)(a.step.wtag >> 32), nst, (int)P2);
+      if (lane == 0) {
+        a.step.next.hdr[2 * cell] = make_int4((int)(uint32_t)a.step.wtag, (int)(uint32_t)(a.step.wtag >> 32), nst, (int)P2);
+        a.step.next.hdr[2 * cell + 1] = make_int4((int)c0, (int)c1, 0, 0);
+      }
     }
   }
   // The window-ring entry the next step reads for this CTA's first stream
@@ -750,6 +752,7 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
         PlanEntry* e = a.step.next.entry + i;
         *reinterpret_cast<int4*>(e) = make_int4(nnew, s + 1, rnext, st / a.hkv);
         e->tag = a.step.wtag;
+        e->first = prefix[i] + s_rank[i];
       }
     }
     for (int v = lane; v < 2 * vec; v += 32) {
@@ -882,7 +885,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   int spec_pg = 0;                     // consumer lanes: page id of the warp's job `lane` in it
   auto load_schedule_head = [&]() {
     const size_t cell = (size_t)tbuf * gridDim.x + blockIdx.x;
-    thdr = ld_early4(a.step.next.hdr + cell);
+    thdr = ld_early4(a.step.next.hdr + 2 * cell);
     if (warp < NCW && warp + NCW * lane < a.step.next.cap)
       spec_pg = ld_early(a.step.next.list + cell * a.step.next.cap + warp + NCW * lane);
   };
@@ -906,15 +909,23 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   // start of this launch with the end of the previous one.
   bool pre_ok = false;     // CTA-uniform: planned and copies issued before the wait
   bool any_miss = true;    // some stream of the call did not match the schedule
+  int pre_k0 = 0, pre_k1 = 0;   // this CTA's range in the guessed plan
+  using Query = typename std::conditional<MMA, MmaQuery<D>, SimtQuery<D>>::type;
+  Query qcur;              // consumer lanes: the query of the piece about to start
+  auto fetch_query = [&](int stream) {
+    if constexpr (MMA) mma_fetch_q<D>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
+    else simt_fetch_q<D, E>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
+  };
   if (STEP && trust != 0 && a.step.pre != 0) {
     load_schedule_head();
+    const int4 trange = ld_early4(a.step.next.hdr + 2 * ((size_t)tbuf * gridDim.x + blockIdx.x) + 1);
     const int status = tid == 0 ? read_status(a.ctrl) : 0;
     const int free_depth = tid == 0 ? *reinterpret_cast<const volatile int32_t*>(&a.ctrl[kCtrlFree]) : 0;
     bool miss = false;
-    int local = 0;
     for (int i = b0; i < e0; ++i) {
       const int4 en = ld_early4(reinterpret_cast<const int4*>(a.step.next.entry + i));
-      const unsigned long long etag = ld_early_u64(&a.step.next.entry[i].tag);
+      const int4 e2 = ld_early4(reinterpret_cast<const int4*>(a.step.next.entry + i) + 1);   // tag, first
+      const unsigned long long etag = (unsigned long long)(uint32_t)e2.x | ((unsigned long long)(uint32_t)e2.y << 32);
       const bool ok = etag == trust && en.w >= 0 && en.w < a.max_seqs;
       const int nn = ok ? en.x : 0;
       s_nold[i] = nn;
@@ -922,15 +933,10 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       s_flag[i] = 0;
       s_rslot[i] = ok && en.y >= a.step.dv.w && (en.z & 1) ? (en.z >> 1) : -1;
       sid[i] = ok ? en.w * a.hkv + i % a.hkv : 0;
-      prefix[i + 1] = (nn + kPage - 1) / kPage;
-      local += prefix[i + 1];
+      // The entries of one step hold the page offsets of its streams, so the
+      // prefix needs no scan (any entry of another step drops the guess).
+      prefix[i + 1] = ok ? e2.z + (nn + kPage - 1) / kPage : 0;
       miss |= !ok;
-    }
-    int total;
-    int run = block_exclusive_scan(local, misc + 3, &total);
-    for (int i = b0; i < e0; ++i) {
-      run += prefix[i + 1];
-      prefix[i + 1] = run;
     }
     if (tid == 0) {
       prefix[0] = 0;
@@ -939,10 +945,10 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     }
     any_miss = __syncthreads_or(miss) != 0;
     const long long P0 = prefix[nst];
-    const long long G0 = P0 < gridDim.x ? P0 : gridDim.x;
-    const int k0 = blockIdx.x < G0 ? (int)(blockIdx.x * P0 / G0) : 0;
-    const int k1 = blockIdx.x < G0 ? (int)((blockIdx.x + 1) * P0 / G0) : 0;
-    pre_ok = misc[1] != 0 && list_matches(P0, k1 - k0, any_miss);
+    const int k0 = trange.x, k1 = trange.y;   // the range the step that wrote the list cut for this CTA
+    pre_ok = misc[1] != 0 && list_matches(P0, k1 - k0, any_miss) && 0 <= k0 && k0 <= k1 && k1 <= P0;
+    pre_k0 = k0;
+    pre_k1 = k1;
     if (pre_ok && warp < NCW) {
       const int nj = k1 - k0 > warp ? (k1 - k0 - warp + NCW - 1) / NCW : 0;
       for (int j = 0; j < spw && j < nj; ++j) {
@@ -965,7 +971,9 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   grid_dependency_wait();
 
   if (pre_ok) {
-    // The call's seq ids against the guess, and the alpha of its new tokens.
+    // The call's seq ids against the guess, and the alpha of its new tokens,
+    // in the same round trip as the query of the CTA's first piece.
+    if (warp < NCW && pre_k1 > pre_k0) fetch_query(stream_of(prefix, nst, pre_k0));
     bool bad = false;
     for (int i = b0; i < e0; ++i) {
       const int seq = a.seq_ids[i / a.hkv];
@@ -979,11 +987,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       // after a landed copy, two on an unused stage), so that each is back at
       // a phase of parity 0 as the pipeline expects; then plan from the seq ids.
       if (warp < NCW && lane == 0) {
-        const long long P0 = prefix[nst];
-        const long long G0 = P0 < gridDim.x ? P0 : gridDim.x;
-        const int k0 = blockIdx.x < G0 ? (int)(blockIdx.x * P0 / G0) : 0;
-        const int k1 = blockIdx.x < G0 ? (int)((blockIdx.x + 1) * P0 / G0) : 0;
-        const int nj = min(spw, k1 - k0 > warp ? (k1 - k0 - warp + NCW - 1) / NCW : 0);
+        const int nj = min(spw, pre_k1 - pre_k0 > warp ? (pre_k1 - pre_k0 - warp + NCW - 1) / NCW : 0);
         for (int j = 0; j < spw; ++j) {
           const uint32_t bar = smem_addr(&full[warp * spw + j]);
           if (j < nj) {
@@ -994,7 +998,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
           mbar_arrive(bar);
         }
       }
-      __syncthreads();   // prefix is read above before the plan below rewrites it
+      __syncthreads();   // every drain is done before the plan below
       pre_ok = false;
     }
   }
@@ -1081,10 +1085,10 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     if (blockIdx.x >= Geff) return;   // uniform over the CTA
   }
   const bool has_range = healthy && blockIdx.x < Geff;
-  const int K0 = has_range ? (int)(blockIdx.x * P / Geff) : 0;
-  const int K1 = has_range ? (int)((blockIdx.x + 1) * P / Geff) : 0;
+  const int K0 = !has_range ? 0 : pre_ok ? pre_k0 : (int)(blockIdx.x * P / Geff);
+  const int K1 = !has_range ? 0 : pre_ok ? pre_k1 : (int)((blockIdx.x + 1) * P / Geff);
   const int ncta = K1 - K0;
-  const bool list_ok = list_matches(P, ncta, any_miss);
+  const bool list_ok = pre_ok || list_matches(P, ncta, any_miss);   // called once: it narrows thdr
   int consumed = 0, issued = 0;
   uint64_t* myfull = full + (warp < NCW ? warp : 0) * spw;
 
@@ -1112,13 +1116,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       return checked(__ldg(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i])));
     };
     using State = typename std::conditional<MMA, MmaState<D>, SimtState<D>>::type;
-    using Query = typename std::conditional<MMA, MmaQuery<D>, SimtQuery<D>>::type;
     State S;
-    Query qcur;
-    auto fetch_query = [&](int stream) {
-      if constexpr (MMA) mma_fetch_q<D>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
-      else simt_fetch_q<D, E>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
-    };
     auto start_piece = [&]() {   // take the fetched query, clear the softmax state
       if constexpr (MMA) mma_start<D>(S, qcur);
       else simt_start<D>(S, qcur);
@@ -1130,14 +1128,14 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     // The first piece's query is requested in the same round trip as the page
     // ids, before the copies fill the memory queues.
     int i = has_range ? stream_of(prefix, nst, K0) : 0;
-    if (has_range) fetch_query(i);
+    if (has_range && !pre_ok) fetch_query(i);   // else fetched with the seq ids
     // STEP: the window-ring entry of every call stream (the token at s - w),
     // requested before the page ids so that both land before the first copies
     // are issued: a load queued behind the grid's first burst of page copies
     // waits microseconds.
     constexpr int kRingPer = (kStepMaxStreams + kMergeThreads - 1) / kMergeThreads;
     int ring_v[STEP ? kRingPer : 1];
-    if constexpr (STEP) {
+    if (STEP && !pre_ok) {   // (the guessed plan knows every leaving slot)
 #pragma unroll
       for (int q = 0; q < kRingPer; ++q) {
         const int il = tid + q * kMergeThreads;
@@ -1160,17 +1158,21 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       if (lane == 0) issue_page<D, MMA, E>(myfull, mystage, spw, j, pg, &tmap, a.kv);
       issued = j + 1;
     };
-    if (pre_ok) issued = min(spw, njobs);   // the first copies went out before the dependency wait
-    else
+    if (pre_ok) {
+      issued = min(spw, njobs);   // the first copies went out before the dependency wait
+    } else {
       for (int j = 0; j < spw && j < njobs; ++j) issue(j);
+    }
     if constexpr (STEP) {
       // The logical slot of the token leaving at this step (-1: none), for the
       // consumers' masks and the step warp's decisions.
+      if (!pre_ok) {
 #pragma unroll
-      for (int q = 0; q < kRingPer; ++q) {
-        const int il = tid + q * kMergeThreads;
-        if (il < nst && s_rslot[il] == kRslotUnknown)
-          s_rslot[il] = (s_pos[il] >= a.step.dv.w && (ring_v[q] & 1)) ? (ring_v[q] >> 1) : -1;
+        for (int q = 0; q < kRingPer; ++q) {
+          const int il = tid + q * kMergeThreads;
+          if (il < nst && s_rslot[il] == kRslotUnknown)
+            s_rslot[il] = (s_pos[il] >= a.step.dv.w && (ring_v[q] & 1)) ? (ring_v[q] >> 1) : -1;
+        }
       }
       named_barrier_arrive(2, kThreads);   // hand them to the step warp (which syncs on barrier 2)
     }

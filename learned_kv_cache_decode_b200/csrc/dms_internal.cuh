@@ -391,15 +391,17 @@ struct __align__(16) PlanEntry {
   int32_t ring;         // window-ring entry of the token that leaves at the next step
   int32_t seq;          // sequence id of call stream i (stream = seq * hkv + i % hkv)
   unsigned long long tag;
-  int32_t pad[2];
+  int32_t first;        // pages of the call streams before stream i (its offset in the range order)
+  int32_t pad;
 };
 // Page list of CTA c for the next step: the physical page ids of its range, in
-// range order, with a header {tag lo, tag hi, call streams, total pages}.
+// range order, with a header of two int4: {tag lo, tag hi, call streams, total
+// pages} and {range begin, range end, 0, 0}.
 // Double-buffered by tag parity: a step reads the buffer of the tag it trusts
 // while it writes the other one.
 struct NextPlan {
   PlanEntry* entry;   // [S]
-  int4* hdr;          // [2][grid]
+  int4* hdr;          // [2][grid][2]
   int32_t* list;      // [2][grid][cap]
   int cap;            // page ids per CTA: enough for any range of any call (max_pages / grid, rounded up)
 };
