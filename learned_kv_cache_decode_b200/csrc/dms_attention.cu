@@ -761,6 +761,24 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
       reinterpret_cast<uint4*>(dv.kv + ((size_t)page * 2 * kPage + (size_t)which * kPage + ts % kPage) * row_bytes)[c] = x;
     }
   }
+
+  // The stream of the range's last piece, when other CTAs hold pieces of it:
+  // if they have all published theirs by now (they are usually done long
+  // before this CTA reaches the end of its range), the consumers will be the
+  // last to finish the stream and can combine without publishing their own
+  // piece and taking a ticket. The acquire read makes the other pieces'
+  // partials visible to them (CTA fence, then the flag).
+  if (lane == 0 && K1 > K0) {
+    const int il = stream_of(prefix, nst, K1 - 1);
+    if (prefix[il] < K0 || prefix[il + 1] > K1) {
+      const long long P = prefix[nst];
+      const long long Geff = P < G ? P : G;
+      const int first = range_of(prefix[il], P, Geff), last = range_of(prefix[il + 1] - 1, P, Geff);
+      const bool done = ld_acquire_gpu(&a.cnt[il]) == last - first;
+      __threadfence_block();
+      *reinterpret_cast<volatile int*>(&misc[3]) = done ? 1 : 2;
+    }
+  }
 }
 
 // One page (16 K rows, then 16 V rows) into a warp's stage j % spw, completing
@@ -842,7 +860,9 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     }
   }
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
-  // misc: [0] abort, [1] ok, [2] last flag, [3 .. 3+warps) scan scratch, [12] free-stack depth
+  // misc: [0] abort, [1] ok, [2] last flag, [3 .. 3+warps) scan scratch (after the plan, STEP:
+  // [3] the other pieces of the range's last stream are all published (1) or not (2), [4] the
+  // consumers' snapshot of [3]), [12] free-stack depth
   // and [13] pages popped by this step (-1: pool exhausted), [14] stream whose combine a split
   // first piece left to the end of the range (-1: none), [15] step decisions ready
   int* misc = reinterpret_cast<int*>(smem + lay.misc);
@@ -1068,6 +1088,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     any_miss = __syncthreads_or(miss) != 0;
   }
   grid_dependents_launch();   // the next kernel may queue up behind this one
+  if (STEP && tid == 0) misc[3] = 0;   // written by the step warp late in the launch
   const bool healthy = misc[1] != 0;
   if constexpr (!STEP) {
     if (!healthy) return;   // poisoned cache: do nothing (uniform over the CTA)
@@ -1247,7 +1268,14 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
         const int inext = pe < K1 ? stream_of(prefix, nst, pe) : i;
         if (pe < K1) load_query(inext);
         const int nn_next = pe < K1 ? retained_of(inext) : 0;
+        // STEP, the range's last piece of a split stream: whether the step warp
+        // has seen every other piece of it published (one snapshot for all).
+        if (STEP && tid == 0 && !whole && pe == K1) misc[4] = *reinterpret_cast<volatile int*>(&misc[3]) == 1;
         named_barrier(1, kMergeThreads);
+        // (read from shared memory where it is used: a register held across the merge spills)
+        auto known_last = [&]() -> bool {
+          return STEP && !whole && pe == K1 && *reinterpret_cast<volatile int*>(&misc[4]) != 0;
+        };
 
         // Merge: thread t owns query head h = t / (D/4) and dims [4 d4, 4 d4 + 4);
         // the CTA's result for its items stays in registers for the combine.
@@ -1285,10 +1313,12 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
             if constexpr (STEP) add_new_token<D, E>(a, i, h, d4, add_new, M, L, O);   // warp-collective
             if (live) store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, L > 0.f ? 1.f / L : 0.f);
           } else if (live) {
-            __stcg(reinterpret_cast<float4*>(&part->O[h][4 * d4]), O);
-            if (d4 == 0) {
-              __stcg(&part->m[h], M);
-              __stcg(&part->l[h], L);
+            if (!known_last()) {   // else nobody reads it: this CTA combines the stream
+              __stcg(reinterpret_cast<float4*>(&part->O[h][4 * d4]), O);
+              if (d4 == 0) {
+                __stcg(&part->m[h], M);
+                __stcg(&part->l[h], L);
+              }
             }
             myO[it] = O;
             myM[it] = M;
@@ -1307,9 +1337,14 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
             // by the whole CTA at the end of the range.
             if (tid == 0 && atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first) misc[14] = i;
           } else {
-            if (tid == 0) misc[2] = (atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first);
-            named_barrier(1, kMergeThreads);
-            if (misc[2]) {
+            const bool shortcut = known_last();
+            if (shortcut) {
+              __threadfence_block();   // the step warp's acquire of the other pieces, passed on
+            } else {
+              if (tid == 0) misc[2] = (atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first);
+              named_barrier(1, kMergeThreads);
+            }
+            if (shortcut || misc[2]) {
               const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
               const int me = blockIdx.x;
 #pragma unroll

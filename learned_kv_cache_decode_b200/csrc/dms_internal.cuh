@@ -314,6 +314,12 @@ __device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
 
 // Acquire-release fence at device scope (weaker and cheaper than the
 // sequentially consistent fence of __threadfence).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 // 64-bit device-scope add with release semantics, no return value.
