@@ -27,6 +27,10 @@ struct dms_cache {
   dms::NextPlan next{};
   uint64_t step_tags = 0;
   uint64_t trust_tag = 0;
+  // Stream lists of the last attention calls ([2][1 + max_seqs], see dms::AttnGuess)
+  // and the number of attention launches so far (its parity picks the buffers).
+  int32_t* attn_guess = nullptr;
+  uint64_t attn_launches = 0;
   int64_t launches = 0;
   bool poisoned = false;   // a device error was observed by dms_get_status
 };
@@ -178,6 +182,8 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
     cudaGetLastError();
   }
   if (e == cudaSuccess && h->has_step) e = alloc_next(dv, h->step_plan.grid, &h->next);
+  if (e == cudaSuccess) e = alloc(&h->attn_guess, (size_t)2 * (1 + c.max_seqs));
+  if (e == cudaSuccess) e = cudaMemset(h->attn_guess, 0xff, (size_t)2 * (1 + c.max_seqs) * sizeof(int32_t));
   const int grid = h->has_step && h->step_plan.grid > h->plan.grid ? h->step_plan.grid : h->plan.grid;
   if (e == cudaSuccess) e = alloc(&dv.part, ((size_t)grid + dv.S) * dms::kMaxGroup * (dv.d + 2));
   if (e == cudaSuccess) e = cudaMemset(dv.kv, 0, (size_t)dv.max_pages * 2 * dms::kPage * dv.d * dv.elem_bytes);
@@ -188,6 +194,7 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
   if (e != cudaSuccess) {
     free_all(dv);
     free_next(h->next);
+    if (h->attn_guess) cudaFree(h->attn_guess);
     delete h;
     cudaGetLastError();
     return e == cudaErrorInvalidValue ? DMS_ERR_INVALID : DMS_ERR_CUDA;
@@ -205,6 +212,7 @@ dms_status dms_cache_destroy(dms_cache* h) {
   cudaError_t e = cudaDeviceSynchronize();
   free_all(h->dv);
   free_next(h->next);
+  if (h->attn_guess) cudaFree(h->attn_guess);
   if (prev >= 0) cudaSetDevice(prev);
   delete h;
   return from_cuda(e);
@@ -235,6 +243,20 @@ dms_status dms_seq_reset(dms_cache* h, cudaStream_t stream, int32_t seq_id) {
 }
 
 namespace {
+
+// dms_decode_attention's launch, with the stream-list guess of the previous
+// attention call on the cache; `early` as recorded for this stream.
+cudaError_t attention_impl(dms_cache* h, cudaStream_t stream, bool early, int32_t n_seqs, const int32_t* seq_ids,
+                           const void* Q, int32_t num_q_heads, float scale, void* out, dms_dtype out_dtype) {
+  const size_t stride = 1 + (size_t)h->cfg.max_seqs;
+  const uint64_t k = h->attn_launches;
+  const dms::AttnGuess guess{h->attn_guess + ((k + 1) & 1) * stride, h->attn_guess + (k & 1) * stride,
+                             early && k > 0};
+  const cudaError_t e = dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
+                                              out_dtype == DMS_F32, guess);
+  if (e == cudaSuccess) h->attn_launches += 1;
+  return e;
+}
 
 dms_status append_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                        const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
@@ -289,9 +311,8 @@ dms_status step_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const in
     h->launches += launches;
     if (e != cudaSuccess) return DMS_ERR_CUDA;
     h->launches += 1;
-    note_launch(h, h->device, stream);
-    return from_cuda(dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
-                                           out_dtype == DMS_F32));
+    note_launch(h, h->device, stream);   // the append just before it writes this cache: no early start
+    return from_cuda(attention_impl(h, stream, false, n_seqs, seq_ids, Q, num_q_heads, scale, out, out_dtype));
   }
   h->launches += 1;
   const uint64_t tag = ++h->step_tags;   // consecutive with trust_tag whenever that is set
@@ -330,9 +351,8 @@ dms_status dms_decode_attention(dms_cache* h, cudaStream_t stream, int32_t n_seq
   if (n_seqs == 0) return DMS_OK;
   if (!seq_ids || !Q || !out || !aligned16(Q) || !aligned16(out)) return DMS_ERR_INVALID;
   h->launches += 1;
-  note_launch(h, h->device, stream);
-  return from_cuda(dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
-                                         out_dtype == DMS_F32));
+  const bool early = note_launch(h, h->device, stream);
+  return from_cuda(attention_impl(h, stream, early, n_seqs, seq_ids, Q, num_q_heads, scale, out, out_dtype));
 }
 
 dms_status dms_decode_step(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,

@@ -74,6 +74,11 @@ struct AttnArgs {
   int spw;      // TMA stages per warp
   int S;        // streams of the cache (sizes the plan arrays in shared memory)
   StepArgs step;   // used by the fused decode-step kernel only
+  // Attention alone: the previous call's stream list (a guess for this call's)
+  // and the buffer this call leaves its own in; plan before the wait when set.
+  const int32_t* guess_rd;
+  int32_t* guess_wr;
+  int pre_attn;
 };
 
 // Largest i in [0, n] with prefix[i] <= x (prefix is non-decreasing, prefix[0] = 0).
@@ -985,21 +990,85 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     }
   }
 
+  // Attention alone, early start: the same idea without a schedule. The
+  // call's streams are guessed to be those of the previous attention call on
+  // this cache (its list is left on the device); their counts, the page table
+  // and the pages are cache state, final before the wait when the kernel before
+  // this one does not write this cache. The guess is checked after the wait.
+  int pid_pre = 0;   // consumer lanes: page id of the warp's job `lane` in the guessed plan
+  if (!STEP && a.pre_attn) {
+    const int status = tid == 0 ? read_status(a.ctrl) : 0;
+    const int gcount = ld_early(a.guess_rd);
+    bool bad = false;
+    int local = 0;
+    for (int i = b0; i < e0; ++i) {
+      const int seq = ld_early(a.guess_rd + 1 + i / a.hkv);   // within the buffer: n_seqs <= max_seqs
+      int pages = 0, st = 0;
+      if (seq < 0 || seq >= a.max_seqs) {
+        bad = true;
+      } else {
+        st = seq * a.hkv + i % a.hkv;
+        pages = (ld_early(a.n + st) + kPage - 1) / kPage;   // through L2: written by earlier launches
+      }
+      sid[i] = st;
+      prefix[i + 1] = pages;
+      local += pages;
+    }
+    int total;
+    int run = block_exclusive_scan(local, misc + 3, &total);
+    for (int i = b0; i < e0; ++i) {
+      run += prefix[i + 1];
+      prefix[i + 1] = run;
+    }
+    if (tid == 0) {
+      prefix[0] = 0;
+      misc[1] = (status == 0);
+    }
+    bad |= gcount != a.n_seqs;
+    pre_ok = !__syncthreads_or(bad) && misc[1] != 0;
+    if (pre_ok) {
+      const long long P0 = prefix[nst];
+      const long long G0 = P0 < gridDim.x ? P0 : gridDim.x;
+      pre_k0 = blockIdx.x < G0 ? (int)(blockIdx.x * P0 / G0) : 0;
+      pre_k1 = blockIdx.x < G0 ? (int)((blockIdx.x + 1) * P0 / G0) : 0;
+      if (warp < NCW) {
+        const int nj = pre_k1 - pre_k0 > warp ? (pre_k1 - pre_k0 - warp + NCW - 1) / NCW : 0;
+        if (lane < nj) {
+          const int kk = pre_k0 + warp + NCW * lane;
+          const int i = stream_of(prefix, nst, kk);
+          pid_pre = ld_early(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i]));
+          if (pid_pre < 0 || pid_pre >= a.max_pages) {
+            latch(a.ctrl, DMS_ERR_INVALID);
+            pid_pre = 0;
+          }
+        }
+        for (int j = 0; j < spw && j < nj; ++j) {
+          const int pg = __shfl_sync(0xffffffffu, pid_pre, j);
+          if (lane == 0)
+            issue_page<D, MMA, E>(full + warp * spw, smem + lay.stages + (size_t)warp * spw * kStage, spw, j, pg,
+                                  &tmap, a.kv);
+        }
+      }
+    }
+  }
+
   // Launched early behind the previous kernel of the stream (programmatic
   // dependent launch): everything above overlaps it; nothing it writes is
   // read before this point.
   grid_dependency_wait();
 
   if (pre_ok) {
-    // The call's seq ids against the guess, and the alpha of its new tokens,
-    // in the same round trip as the query of the CTA's first piece.
+    // The call's seq ids against the guess, and (STEP) the alpha of its new
+    // tokens, in the same round trip as the query of the CTA's first piece.
     if (warp < NCW && pre_k1 > pre_k0) fetch_query(stream_of(prefix, nst, pre_k0));
     bool bad = false;
     for (int i = b0; i < e0; ++i) {
       const int seq = a.seq_ids[i / a.hkv];
-      const int al = alpha_at(a.step.asrc, (size_t)(i / a.hkv), i % a.hkv);
+      if constexpr (STEP) {
+        const int al = alpha_at(a.step.asrc, (size_t)(i / a.hkv), i % a.hkv);
+        s_flag[i] = al != 0 ? 2 : 0;
+      }
       bad |= seq != sid[i] / a.hkv;
-      s_flag[i] = al != 0 ? 2 : 0;
     }
     if (__syncthreads_or(bad)) {
       // Another call: let the guessed copies land, then take every stage
@@ -1089,6 +1158,10 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   }
   grid_dependents_launch();   // the next kernel may queue up behind this one
   if (STEP && tid == 0) misc[3] = 0;   // written by the step warp late in the launch
+  if (!STEP && a.guess_wr && blockIdx.x == 0) {   // this call's stream list, the next call's guess
+    for (int b = tid; b < a.n_seqs; b += kThreads) a.guess_wr[1 + b] = a.seq_ids[b];
+    if (tid == 0) a.guess_wr[0] = a.n_seqs;
+  }
   const bool healthy = misc[1] != 0;
   if constexpr (!STEP) {
     if (!healthy) return;   // poisoned cache: do nothing (uniform over the CTA)
@@ -1166,7 +1239,9 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       }
     }
     int jb = 0;   // page ids of jobs [jb, jb+32) in pid_cur, [jb+32, jb+64) in pid_nxt
-    int pid_cur = (STEP && list_ok) ? (lane < njobs ? checked(spec_pg) : 0) : lookup(lane);
+    int pid_cur = (STEP && list_ok) ? (lane < njobs ? checked(spec_pg) : 0)
+                  : (!STEP && pre_ok) ? pid_pre   // looked up before the wait
+                                      : lookup(lane);
     int pid_nxt = lookup(32 + lane);
     auto issue = [&](int j) {   // warp-uniform; j = issued
       if (j - jb >= 32) {
@@ -1534,9 +1609,12 @@ AttnArgs attn_args(const Dev& dv, const AttnPlan& plan, int n_seqs, const int32_
 
 cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,
                              const int32_t* seq_ids, const void* Q, int hq, float scale, void* out,
-                             int out_f32) {
+                             int out_f32, const AttnGuess& guess) {
   if (n_seqs == 0) return cudaSuccess;
-  const AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32);
+  AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32);
+  a.guess_rd = guess.rd;
+  a.guess_wr = guess.wr;
+  a.pre_attn = guess.early && guess.rd && guess.wr ? 1 : 0;
   return launch_dependent(reinterpret_cast<KernelFn>(plan.fn), dim3(plan.grid), dim3(plan.threads), plan.smem, st,
                           a, plan.tmap);
 }

@@ -421,8 +421,19 @@ cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, in
                         bool early);
 constexpr int kStepMaxStreams = 1024;   // caches with more streams run the step as two launches
 
+// The stream list of the previous attention call on a cache, kept on the device
+// as a guess for the next one: [2][1 + max_seqs] ints, {n_seqs, seq ids...} per
+// parity (a launch reads one buffer while it writes the other). `early`: the
+// host knows that the kernel just before this launch in its stream does not
+// write this cache, so the launch may plan from the guess and the cache state
+// and start its first page copies before its dependency wait (checked after it).
+struct AttnGuess {
+  const int32_t* rd;   // the previous call's list (count < 0: none)
+  int32_t* wr;         // this call's list, for the next call
+  bool early;
+};
 cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,
                              const int32_t* seq_ids, const void* Q, int hq, float scale, void* out,
-                             int out_f32);
+                             int out_f32, const AttnGuess& guess);
 
 }  // namespace dms

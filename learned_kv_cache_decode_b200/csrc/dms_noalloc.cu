@@ -126,6 +126,6 @@ extern "C" dms_status dms_decode_attention_noalloc(cudaStream_t stream, const dm
   // error may not. The partials are written before they are read.
   if (cudaMemsetAsync(scratch, 0, kCtrlBytes + (size_t)nst * 4, stream) != cudaSuccess) return DMS_ERR_CUDA;
   cudaError_t e = launch_attention(dv, plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
-                                   out_dtype == DMS_F32);
+                                   out_dtype == DMS_F32, AttnGuess{nullptr, nullptr, false});
   return e == cudaSuccess ? DMS_OK : DMS_ERR_CUDA;
 }

@@ -359,6 +359,54 @@ def test_fused_step_schedule_follows_every_change(case, caches):
             run.close()
 
 
+GUESS_CASES = [
+    wl("guess-bf16-g7-d128", 6, 14, 2, 128, "bf16", 8, (1, 500), 0, 0.6, 38),
+    wl("guess-f32-g4-d64", 5, 8, 2, 64, "f32", 24, (1, 400), 0, 0.5, 39),
+]
+
+
+@pytest.mark.parametrize("case", GUESS_CASES, ids=[c.name for c in GUESS_CASES])
+def test_attention_alone_guess_follows_every_change(case):
+    """dms_decode_attention on two caches, back to back after all of a step's appends:
+    the kernel before each attention launch is the other cache's, so the launch guesses
+    its stream list from the previous attention call on its cache, plans from the cache
+    state and starts its first copies before its dependency wait, then checks the guess
+    against the seq ids. The attention lists change from call to call (the same, a
+    permutation, a subset, a superset, twice on the same state); every output against
+    the oracle."""
+    B = case.batch
+    every = list(range(B))
+    perm = [3, 1, 0, 4, 2] + list(range(5, B))
+    lists = [[every, every], [every], [perm], [perm, perm], [perm[:3]], [every, every[::-1]], [every], [every]]
+    runs = [Run(case, steps=len(lists)) for _ in range(2)]
+    tol = dict(max_abs=1e-4, mean_abs=1e-5) if case.dtype == "f32" else {}
+    try:
+        for run in runs:
+            run.prefill(chunk=97)
+        for step, calls in enumerate(lists):
+            for run in runs:   # one token for every sequence of both caches first
+                K, V, A, _ = run.decode_inputs(step, every)
+                run.cache.append(torch.tensor(every, dtype=torch.int32, device="cuda"), to_device(K, case),
+                                 to_device(V, case), torch.from_numpy(A).cuda())
+                assert run.sim.append(every, [1] * B, A)[0] == 0
+                for b in every:
+                    run.seen[b] += 1
+            for seqs in calls:   # then the attention calls, alternating between the caches
+                Qall = W.query(case, step)
+                outs = [run.cache.decode_attention(torch.tensor(seqs, dtype=torch.int32, device="cuda"),
+                                                   to_device(Qall[seqs], case), scale=run.scale) for run in runs]
+                torch.cuda.synchronize()
+                for run, out in zip(runs, outs):
+                    for j, b in enumerate(seqs):
+                        compare(out[j], run.oracle_out(b, Qall[b]), **tol)
+        for run in runs:
+            run.check_metadata()
+            assert run.cache.status() == _native.DMS_OK
+    finally:
+        for run in runs:
+            run.close()
+
+
 def test_decode_step_captured_in_a_cuda_graph_replays_step_after_step():
     """dms_decode_step captured into a CUDA graph (issued as dms_append +
     dms_decode_attention under capture), replayed once per decode step with the
