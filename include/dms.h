@@ -153,7 +153,14 @@ dms_status dms_append_keyed(dms_cache* cache, cudaStream_t stream, int32_t n_seq
  *   num_q_heads  host int; a multiple of num_kv_heads with g <= 8
  *   scale        host float (usually 1 / sqrt(head_dim))
  *   out          device [n_seqs, num_q_heads, head_dim] of out_dtype
- * A stream with no tokens yields zeros. Async. */
+ * A stream with no tokens yields zeros.
+ * Each call leaves its stream list on the device for the next call on the
+ * cache. When the kernel just before a call in its stream is not one of this
+ * cache's, the call guesses that it has the previous call's streams. It plans
+ * from the cache state and starts its first page copies before that kernel has
+ * finished (programmatic dependent launch), and checks the guess against
+ * seq_ids once it has. Calls on one cache must run in the order they are made:
+ * on one stream, or on streams ordered by events. Async. */
 dms_status dms_decode_attention(dms_cache* cache, cudaStream_t stream, int32_t n_seqs,
                                 const int32_t* seq_ids, const void* Q, int32_t num_q_heads,
                                 float scale, void* out, dms_dtype out_dtype);
