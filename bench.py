@@ -170,15 +170,24 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def code_fingerprint(path: str) -> str:
+    """sha256 of a C++/CUDA source with its comments and whitespace removed: it
+    changes with the code, not with the comments."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return hashlib.sha256(re.sub(r"\s+", "", text).encode()).hexdigest()
+
+
 def profile_traffic(workload: str, kernel: str, entry: str = "dms_decode_attention"):
     """Per-launch DRAM bytes of the timed kernel from the committed ncu summary,
-    valid only while the kernel source is unchanged since the capture."""
+    valid only while the kernel code is unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", f"{entry}_{kernel}_{workload}.md")
     src = os.path.join(ROOT, "learned_kv_cache_decode_b200", "csrc", "dms_attention.cu")
     try:
         text = open(path).read()
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+        sha = code_fingerprint(src)
+        m_sha = re.search(r"code_sha256:\s*([0-9a-f]{64})", text)
         m_tr = re.search(r"traffic_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
         if m_sha and m_tr and m_sha.group(1) == sha:
             return float(m_tr.group(1))

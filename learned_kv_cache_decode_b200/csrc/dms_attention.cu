@@ -10,10 +10,13 @@
 //  * Persistent grid. The call's retained pages, concatenated stream after
 //    stream, are cut into equal contiguous ranges, one per CTA (split-K with
 //    exact balance whatever the per-stream lengths are). Every CTA derives
-//    the plan itself from the retained counts: no host sync, no extra launch.
-//  * One producer warp issues TMA copies of whole pages (K rows and V rows
-//    are contiguous in a page) into a ring of shared-memory stages guarded by
-//    mbarriers; consumer warps take pages round-robin.
+//    the plan itself on the device: no host sync, no extra launch. A fused
+//    step inherits it from the step before (a schedule), and a launch whose
+//    previous kernel in the stream belongs to another cache plans and starts
+//    its first copies before its dependency wait.
+//  * Every warp runs its own page pipeline: it issues TMA copies of whole
+//    pages (K rows and V rows are contiguous in a page) into its own ring of
+//    shared-memory stages guarded by mbarriers, and computes on them in order.
 //  * Page compute, two variants:
 //      MMA  - S^T = K_page (16 x d) * Q^T (d x 8): one m16n8k16 row of tiles
 //             per page, the GQA group padded to 8 columns; fp32 online
