@@ -519,6 +519,8 @@ __device__ __forceinline__ void combine_stream(const AttnArgs& a, int i, int fir
     const bool live = t < items;
     if (!__any_sync(0xffffffffu, live)) break;   // warp-uniform
     const int h = (live ? t : 0) / (D / 4), d4 = (live ? t : 0) % (D / 4);
+    NewTok nt;
+    if constexpr (STEP) fetch_new_token<D, E>(a, i, h, d4, nt);   // in flight with the partials
     float M = -INFINITY, L = 0.f;
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
@@ -536,7 +538,7 @@ __device__ __forceinline__ void combine_stream(const AttnArgs& a, int i, int fir
       for (int u = 0; u < 4; ++u)
         if (c0 + u <= last) merge_into(M, L, O, mc[u], lc[u], oc[u]);
     }
-    if constexpr (STEP) add_new_token<D, E>(a, i, h, d4, add_new, M, L, O);   // warp-collective
+    if constexpr (STEP) apply_new_token<D>(nt, a.sl2e, add_new, M, L, O);   // warp-collective
     if (live) store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, L > 0.f ? 1.f / L : 0.f);
   }
 }
@@ -1360,8 +1362,12 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
         constexpr int kItems = kMaxGroup * D / 4;
         constexpr int kIters = (kItems + kMergeThreads - 1) / kMergeThreads;
         const int items = a.g * (D / 4);
-        if (STEP) await_decisions();
-        const bool add_new = STEP && s_tslot[i] >= 0;   // the stream's new token (appended by this step)
+        // The step warp's decisions are needed only by a merge that may finish
+        // its stream (a whole piece, or the range's last piece, which may
+        // combine); a split first piece only publishes its partial.
+        const bool may_finish = whole || pe == K1;
+        if (STEP && may_finish) await_decisions();
+        const bool add_new = STEP && may_finish && s_tslot[i] >= 0;   // the stream's new token (appended by this step)
         float4 myO[kIters];
         float myM[kIters], myL[kIters];
         Partial<D>* part = reinterpret_cast<Partial<D>*>(a.part) + (blockIdx.x + i);
@@ -1431,6 +1437,8 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
                 const bool live = t < items;
                 if (!__any_sync(0xffffffffu, live)) break;   // warp-uniform
                 const int h = (live ? t : 0) / (D / 4), d4 = (live ? t : 0) % (D / 4);
+                NewTok nt;   // tensor-core kernel: in flight with the partials (the CUDA-core one has no registers to spare)
+                if constexpr (STEP && MMA) fetch_new_token<D, E>(a, i, h, d4, nt);
                 float M = live ? myM[it] : 0.f, L = live ? myL[it] : 1.f;
                 float4 O = live ? myO[it] : make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
@@ -1448,7 +1456,8 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
 #pragma unroll
                   for (int u = 0; u < 4; ++u) merge_into(M, L, O, mc[u], lc[u], oc[u]);
                 }
-                if constexpr (STEP) add_new_token<D, E>(a, i, h, d4, add_new, M, L, O);   // warp-collective
+                if constexpr (STEP && MMA) apply_new_token<D>(nt, a.sl2e, add_new, M, L, O);   // warp-collective
+                else if constexpr (STEP) add_new_token<D, E>(a, i, h, d4, add_new, M, L, O);
                 if (live) store_out4(a, b, kvh * a.g + h, 4 * d4, D, O, L > 0.f ? 1.f / L : 0.f);
               }
               if (tid == 0) a.cnt[i] = 0;   // ready for the next launch (stream order)
