@@ -190,6 +190,10 @@ dms_status dms_decode_attention(dms_cache* cache, cudaStream_t stream, int32_t n
  * its seq ids are those of the step that left the schedule; the guess is
  * checked once the previous kernel is done. Calls on one cache must run in
  * the order they are made: on one stream, or on streams ordered by events.
+ * Every kernel of this library that writes a cache lets the next kernel of its
+ * stream start only after its own dependency wait; other code that uses
+ * programmatic dependent launch on the same stream must do the same (call
+ * cudaGridDependencySynchronize before cudaTriggerProgrammaticLaunchCompletion).
  *   n_seqs, seq_ids      as dms_append (one token per sequence)
  *   K, V                 device [n_seqs, num_kv_heads, head_dim] of the cache dtype, 16-B aligned
  *   alpha                device uint8 [n_seqs, num_kv_heads]

@@ -40,11 +40,14 @@ namespace {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // The cache whose kernels were launched last on each stream. Kernels that
-// write a cache are launched only through these calls, so when the record of a
-// stream names another cache, the kernel just before the next launch on that
-// stream (this library's or anyone's) does not write this one. A stream with
-// no record, or one whose record was evicted, counts as this cache's. The
-// per-thread default stream is a different stream in every host thread.
+// write a cache are launched only through these calls, and each lets the next
+// kernel of its stream start only after its own dependency wait. So when the
+// record of a stream names another cache, no kernel still running ahead of the
+// next launch on that stream writes this one. The stats kernel, which writes
+// no cache state and lets the next kernel start at once, is not recorded. A
+// stream with no record, or one whose record was evicted, counts as this
+// cache's. The per-thread default stream is a different stream in every host
+// thread.
 struct StreamLast {
   int device;
   cudaStream_t stream;
@@ -373,7 +376,8 @@ dms_status dms_stats(dms_cache* h, cudaStream_t stream, int32_t* retained, int32
   if (!h) return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
   h->launches += 1;
-  note_launch(h, h->device, stream);
+  // Not recorded: the stats kernel writes no cache state and lets the next
+  // kernel start at once (see dms::grid_dependents_launch).
   return from_cuda(dms::launch_stats(h->dv, stream, retained, seen, head_cr, totals));
 }
 

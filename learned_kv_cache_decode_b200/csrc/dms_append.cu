@@ -409,8 +409,9 @@ __global__ void init_state_kernel(Dev dv) {
 __global__ void __launch_bounds__(256)
 stats_kernel(Dev dv, int32_t* retained, int32_t* seen, float* head_cr, int64_t* totals) {
   // Launched behind the previous kernel of the stream (programmatic dependent
-  // launch). The kernel after this one may start at once: what it reads before
-  // its own dependency wait is nothing this kernel writes.
+  // launch). It writes no cache state, so the kernel after it may start at
+  // once; the host leaves it out of its per-stream record of the last cache
+  // launched (see grid_dependents_launch).
   grid_dependents_launch();
   __shared__ unsigned long long s_head[kMaxKvHeads][2];
   for (int h = threadIdx.x; h < dv.hkv; h += blockDim.x) s_head[h][0] = s_head[h][1] = 0;

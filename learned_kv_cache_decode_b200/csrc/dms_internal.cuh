@@ -279,6 +279,14 @@ __device__ __forceinline__ unsigned long long ld_early_u64(const unsigned long l
 // must call grid_dependency_wait() before it touches memory that earlier
 // work writes or reads. grid_dependents_launch() lets the next such kernel
 // start launching; it never weakens that kernel's own wait.
+// Every kernel of this library that writes a cache's state or scratch calls
+// grid_dependents_launch() only after its own grid_dependency_wait(), and the
+// host records it as the last cache launched on its stream. The stats kernel
+// writes neither: it triggers at once and is not recorded. So when a kernel
+// starts, every kernel before the last recorded one ahead of it in the stream
+// has completed, and that one belongs to the recorded cache. The early starts
+// of the attention and fused-step kernels rely on this: they read their
+// cache's state before their wait when the record names another cache.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 

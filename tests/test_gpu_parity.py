@@ -359,6 +359,30 @@ def test_fused_step_schedule_follows_every_change(case, caches):
             run.close()
 
 
+def test_fused_step_after_another_caches_stats_kernel():
+    """Fused steps on cache A with a dms_stats call on cache B between them. The stats
+    kernel lets the next kernel start at once, so A's previous step may still be running
+    when the next one starts; the host leaves stats out of its per-stream record, so the
+    record still names A and the step does not read A's state before its wait.
+    Metadata and every output against the oracle."""
+    case = wl("after-stats-bf16-g7-d128", 4, 14, 2, 128, "bf16", 8, (40, 500), 12, 0.6, 40)
+    a, b = Run(case), Run(case)
+    try:
+        a.prefill(chunk=97)
+        b.prefill(chunk=97)
+        for step in range(case.decode_steps):
+            out, Q = a.decode_step(step, fused=True)
+            b.cache.stats()
+            torch.cuda.synchronize()
+            for j in range(case.batch):
+                compare(out[j], a.oracle_out(j, Q[j]))
+        a.check_metadata()
+        assert a.cache.status() == _native.DMS_OK and b.cache.status() == _native.DMS_OK
+    finally:
+        a.close()
+        b.close()
+
+
 GUESS_CASES = [
     wl("guess-bf16-g7-d128", 6, 14, 2, 128, "bf16", 8, (1, 500), 0, 0.6, 38),
     wl("guess-f32-g4-d64", 5, 8, 2, 64, "f32", 24, (1, 400), 0, 0.5, 39),
