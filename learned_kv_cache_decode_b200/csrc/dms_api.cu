@@ -60,8 +60,16 @@ StreamLast g_last[kStreamRecords];
 int g_last_next = 0;
 
 // Records `c` as the last cache launched on `s`; returns true when the
-// previous record of `s` named another cache.
+// previous record of `s` named another cache. A launch into a stream being
+// captured into a graph runs later, if at all, so it is neither recorded nor
+// started early (a graph launch waits for the work before it in its stream).
 bool note_launch(const dms_cache* c, int device, cudaStream_t s) {
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &capture) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (capture != cudaStreamCaptureStatusNone) return false;
   const std::thread::id th = s == cudaStreamPerThread ? std::this_thread::get_id() : std::thread::id();
   std::lock_guard<std::mutex> lock(g_last_mu);
   for (StreamLast& e : g_last) {

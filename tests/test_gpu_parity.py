@@ -473,6 +473,54 @@ def test_decode_step_captured_in_a_cuda_graph_replays_step_after_step():
         run.close()
 
 
+def test_attention_of_two_caches_captured_in_a_graph_between_eager_calls():
+    """dms_decode_attention on two caches captured into one CUDA graph, replayed once
+    per step after eager appends, with eager attention calls on the same stream between
+    replays. Launches into a capturing stream are neither recorded nor started early, so
+    the eager calls' early starts see only what really ran. Every output against the
+    oracle."""
+    case = wl("graph-two-caches", 4, 14, 2, 128, "bf16", 8, (40, 500), 6, 0.6, 41)
+    runs = [Run(case), Run(case)]
+    B = case.batch
+    every = list(range(B))
+    ids = torch.tensor(every, dtype=torch.int32, device="cuda")
+    try:
+        for run in runs:
+            run.prefill(chunk=97)
+        dQ = [torch.empty((B, case.num_q_heads, case.head_dim), dtype=torch.bfloat16, device="cuda")
+              for _ in runs]
+        outs = [torch.empty_like(q) for q in dQ]
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for run, q, o in zip(runs, dQ, outs):
+                run.cache.decode_attention(ids, q, scale=run.scale, out=o)
+        for step in range(case.decode_steps):
+            Q = W.query(case, step)
+            for run, q in zip(runs, dQ):
+                K, V, A, _ = run.decode_inputs(step, every)
+                run.cache.append(ids, to_device(K, case), to_device(V, case), torch.from_numpy(A).cuda())
+                assert run.sim.append(every, [1] * B, A)[0] == 0
+                for b in every:
+                    run.seen[b] += 1
+                q.copy_(to_device(Q, case))
+            g.replay()
+            eager = [run.cache.decode_attention(ids, to_device(Q, case), scale=run.scale) for run in runs]
+            torch.cuda.synchronize()
+            for run, o, e in zip(runs, outs, eager):
+                for b in every:
+                    ref = run.oracle_out(b, Q[b])
+                    compare(o[b], ref)
+                    compare(e[b], ref)
+        for run in runs:
+            run.check_metadata()
+            assert run.cache.status() == _native.DMS_OK
+        del g
+    finally:
+        for run in runs:
+            run.close()
+
+
 # ---------------------------------------------------------------------------
 # alpha read from a designated key channel (dms_append_keyed, dms_decode_step_keyed)
 
