@@ -359,6 +359,31 @@ def test_fused_step_schedule_follows_every_change(case, caches):
             run.close()
 
 
+SWEEP_WINDOWS = [1, 2, 16, 32, 64, 128, 256]
+
+
+@pytest.mark.parametrize("w", SWEEP_WINDOWS)
+@pytest.mark.parametrize("fused", [False, True], ids=["two_launches", "fused_step"])
+def test_window_sweep(w, fused):
+    """The delayed-eviction window swept from immediate eviction (w = 1, reading R15) to
+    256, on one workload shape, through both decode paths: metadata bit for bit, every
+    output against the oracle."""
+    case = wl(f"sweep-w{w}", 3, 21, 3, 128, "bf16", w, (300, 900), 6, 0.7, 42)
+    run = Run(case)
+    try:
+        run.prefill(chunk=257)
+        run.check_metadata()
+        for step in range(case.decode_steps):
+            out, Q = run.decode_step(step, fused=fused)
+            torch.cuda.synchronize()
+            for b in range(case.batch):
+                compare(out[b], run.oracle_out(b, Q[b]))
+        run.check_metadata()
+        assert run.cache.status() == _native.DMS_OK
+    finally:
+        run.close()
+
+
 def test_fused_step_after_another_caches_stats_kernel():
     """Fused steps on cache A with a dms_stats call on cache B between them. The stats
     kernel lets the next kernel start at once, so A's previous step may still be running
