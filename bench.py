@@ -59,6 +59,10 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--depth", default="",
+                    help="CR_FIRST,CR_LAST: compression growing with depth, each layer cache with its "
+                         "own alpha rate (workloads.depth_layers); per-layer dms_stats at every step; "
+                         "no e2e pass")
     return ap.parse_args()
 
 
@@ -301,6 +305,9 @@ def main():
     if args.window:
         import dataclasses
         wl = dataclasses.replace(wl, window=args.window)
+    depth = [float(x) for x in args.depth.split(",")] if args.depth else None
+    if depth:
+        args.no_e2e = True   # the e2e pass copies one alpha row per step for all layers
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         run_reference(args, wl, world, rank)
@@ -335,24 +342,35 @@ def main():
     d_cu = torch.from_numpy(offs.astype(np.int32)).to(dev)
     ids = torch.arange(B, dtype=torch.int32, device=dev)   # cache-local sequence ids
 
-    def new_layer(max_pages):
+    def new_layer(max_pages, alpha):
         c = DmsCache(B, hkv, d, wl.window, max_pages, mps, dtype=tdt, attn_kernel=args.attn_kernel)
-        c.append(ids, dK, dV, dA, cu_tokens=d_cu)
+        c.append(ids, dK, dV, alpha, cu_tokens=d_cu)
         return c
 
-    # Probe cache (worst-case pool) to learn the retained counts, then size every
-    # layer pool to what the prompt keeps plus room for every decode token.
-    probe = new_layer(B * hkv * mps)
-    st0 = probe.stats()
-    torch.cuda.synchronize()
-    retained = st0["retained"].cpu().numpy().astype(np.int64)
-    retained0 = int(retained.sum())
-    probe.close()
-    del probe
-    pool = int(((retained + 15) // 16).sum()) + B * hkv * (n_dec // 16 + 2)
-    layer_bytes = retained0 * d * 2 * wl.elem_bytes
-    L = args.layers or max(1, min(32, math.ceil(8 * L2_BYTES / max(layer_bytes, 1))))
-    caches = [new_layer(pool) for _ in range(L)]
+    if depth:
+        # One alpha stream per layer (compression growing with depth); worst-case pools.
+        L = args.layers or 8
+        layer_wls = W.depth_layers(wl, L, depth[0], depth[-1])
+        pool = B * hkv * mps
+        caches, A_first = [], None
+        for lw in layer_wls:
+            a_l = np.concatenate([W.alpha(lw, b, 0, int(c_)) for b, c_ in zip(seqs, ctx)])
+            A_first = a_l if A_first is None else A_first
+            caches.append(new_layer(pool, torch.from_numpy(a_l).to(dev)))
+    else:
+        # Probe cache (worst-case pool) to learn the retained counts, then size every
+        # layer pool to what the prompt keeps plus room for every decode token.
+        probe = new_layer(B * hkv * mps, dA)
+        st0 = probe.stats()
+        torch.cuda.synchronize()
+        retained = st0["retained"].cpu().numpy().astype(np.int64)
+        retained0 = int(retained.sum())
+        probe.close()
+        del probe
+        pool = int(((retained + 15) // 16).sum()) + B * hkv * (n_dec // 16 + 2)
+        layer_bytes = retained0 * d * 2 * wl.elem_bytes
+        L = args.layers or max(1, min(32, math.ceil(8 * L2_BYTES / max(layer_bytes, 1))))
+        caches = [new_layer(pool, dA) for _ in range(L)]
     torch.cuda.synchronize()
     del dK, dV, dA
     torch.cuda.empty_cache()
@@ -362,9 +380,14 @@ def main():
 
     # decode-step inputs: device-resident for the timed pass, pinned host for the e2e pass
     Kd, Vd, Ad, Qd = host_decode(wl, seqs, ctx, n_dec)
+    if depth:   # [L, steps, B, Hkv]: every layer its own decisions
+        Ad = np.stack([np.stack([W.alpha(lw, b, int(c_), n_dec) for b, c_ in zip(seqs, ctx)], axis=1)
+                       for lw in layer_wls])
     t_K, t_V, t_A, t_Q = (to_torch(x, dev) for x in (Kd, Vd, Ad, Qd))
     outs = [torch.empty((B, hq, d), dtype=tdt, device=dev) for _ in range(L)]
-    totals = torch.zeros((n_dec, 2), dtype=torch.int64, device=dev)
+    # (seen, retained) totals after every step: of layer 0 (every layer holds the same
+    # tokens), or of every layer with --depth
+    totals = torch.zeros((n_dec, L if depth else 1, 2), dtype=torch.int64, device=dev)
 
     lib = caches[0].lib
     hs = [c._h for c in caches]
@@ -383,23 +406,28 @@ def main():
     fused = args.step == "fused"
     odt = 0 if tdt == torch.bfloat16 else 1
 
+    def alpha_ptr(t, l):
+        return pA + ((l * n_dec if depth else 0) + t) * B * hkv
+
     def step(t, timed):
         for l in range(L):
             h = hs[l]
             rc = 0
             if not fused:
-                rc |= lib.dms_append(h, sp, B, pids, None, B, pK + t * row_kv, pV + t * row_kv, pA + t * B * hkv)
+                rc |= lib.dms_append(h, sp, B, pids, None, B, pK + t * row_kv, pV + t * row_kv, alpha_ptr(t, l))
             if timed:
                 e0, e1 = ev_pairs[(t - t_pl) * L + l]
                 e0.record(stream)
             if fused:
-                rc |= lib.dms_decode_step(h, sp, B, pids, pK + t * row_kv, pV + t * row_kv, pA + t * B * hkv,
+                rc |= lib.dms_decode_step(h, sp, B, pids, pK + t * row_kv, pV + t * row_kv, alpha_ptr(t, l),
                                           pQ + t * row_q, hq, scale, outs[l].data_ptr(), odt)
             else:
                 rc |= lib.dms_decode_attention(h, sp, B, pids, pQ + t * row_q, hq, scale, outs[l].data_ptr(), odt)
             if timed:
                 e1.record(stream)
-            if l == 0:   # every layer holds the same tokens: one stats call gives the bytes of all
+            if depth:   # every layer its own retained set
+                rc |= lib.dms_stats(h, sp, None, None, None, pT + (t * L + l) * 16)
+            elif l == 0:   # every layer holds the same tokens: one stats call gives the bytes of all
                 rc |= lib.dms_stats(h, sp, None, None, None, pT + t * 16)
             if rc:
                 raise RuntimeError(f"library call failed ({rc})")
@@ -428,16 +456,16 @@ def main():
     for t in range(t_pl, t_pl + args.steps):
         step(t, True)
     torch.cuda.synchronize()
-    tot = totals.cpu().numpy()
-    timed_tot = tot[args.warmup:args.warmup + args.steps]           # [steps, 2]
-    bytes_launch = np.repeat(timed_tot[:, 1:2].astype(np.float64), L, axis=1) * d * 2 * wl.elem_bytes
+    tot = totals.cpu().numpy()                                         # [steps, 1 or L, 2]
+    per_layer = tot if depth else np.repeat(tot, L, axis=1)            # [steps, L, 2]
+    timed_tot = per_layer[args.warmup:args.warmup + args.steps].sum(axis=1)   # [steps, 2] over layers
+    bytes_launch = per_layer[args.warmup:args.warmup + args.steps, :, 1].astype(np.float64) * d * 2 * wl.elem_bytes
     total_bytes = float(bytes_launch.sum())
     same = [c.stats()["totals"].cpu().numpy().tolist() for c in caches]
-    if any(x != same[0] for x in same):
+    if not depth and any(x != same[0] for x in same):
         raise RuntimeError(f"layer caches diverged: {same}")
     attn_ms = np.array([a.elapsed_time(b) for a, b in ev_pairs])
-    pl_tot = tot[t_pl:t_pl + args.steps]
-    bytes_pl = np.repeat(pl_tot[:, 1:2].astype(np.float64), L, axis=1) * d * 2 * wl.elem_bytes
+    bytes_pl = per_layer[t_pl:t_pl + args.steps, :, 1].astype(np.float64) * d * 2 * wl.elem_bytes
     status = [c.status() for c in caches]
     if any(status):
         raise RuntimeError(f"device status {status}")
@@ -462,7 +490,7 @@ def main():
     else:
         for t in range(t_b, t_b + burst_steps):   # keep the decode going: append outside the events
             for l in range(L):
-                lib.dms_append(hs[l], sp, B, pids, None, B, pK + t * row_kv, pV + t * row_kv, pA + t * B * hkv)
+                lib.dms_append(hs[l], sp, B, pids, None, B, pK + t * row_kv, pV + t * row_kv, alpha_ptr(t, l))
             lib.dms_stats(hs[0], sp, None, None, None, pT + t * 16)
         e_b0.record(stream)
         for t in range(t_b, t_b + burst_steps):
@@ -471,8 +499,8 @@ def main():
         e_b1.record(stream)
     torch.cuda.synchronize()
     burst_ms = e_b0.elapsed_time(e_b1) / (burst_steps * L)
-    b_tot = totals.cpu().numpy()[t_b:t_b + burst_steps]
-    achieved_burst = float(b_tot[:, 1].astype(np.float64).mean()) * d * 2 * wl.elem_bytes / (burst_ms * 1e-3) / 1e9
+    b_tot = totals.cpu().numpy()[t_b:t_b + burst_steps]   # [steps, 1 or L, 2]
+    achieved_burst = float(b_tot[:, :, 1].astype(np.float64).mean()) * d * 2 * wl.elem_bytes / (burst_ms * 1e-3) / 1e9
     # Roofline of the dominant kernel. Fused: the timed region holds the step
     # launches, back to back as a decode loop issues them, plus one small
     # dms_stats launch per step, so its average launch duration is this rank's
@@ -556,7 +584,7 @@ def main():
         e_b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e_a.elapsed_time(e_b)
-        tot2 = totals.cpu().numpy()[t0_e2e:t0_e2e + args.steps]
+        tot2 = totals.cpu().numpy()[t0_e2e:t0_e2e + args.steps, 0]   # layer 0 stands for all (no --depth)
         e2e_bytes = float(tot2[:, 1].astype(np.float64).sum()) * L * d * 2 * wl.elem_bytes
         e2e_ms, e2e_bytes = reduce_over_ranks(e2e_ms, e2e_bytes, world, dev)
         h2d_b = 2 * row_kv + B * hkv + row_q
@@ -569,9 +597,10 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sample_seqs = list(range(min(B, 2)))
+        A_s, Ad_s = (A_first, Ad[0]) if depth else (A_p, Ad)   # --depth: layer 0's decisions
         items, nbytes = oracle_sample(wl, [seqs[i] for i in sample_seqs], args.warmup + args.steps,
-                                      (K_p, V_p, A_p, offs),
-                                      (Kd[:, sample_seqs], Vd[:, sample_seqs], Ad[:, sample_seqs],
+                                      (K_p, V_p, A_s, offs),
+                                      (Kd[:, sample_seqs], Vd[:, sample_seqs], Ad_s[:, sample_seqs],
                                        Qd[:, sample_seqs]))
         reps, t_cpu, threads = time_oracle(items, wl.window, scale, args.cpu_seconds)
         cpu = {"value": nbytes * reps / t_cpu / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
@@ -588,14 +617,18 @@ def main():
                 "workload": wl.name, "batch_per_gpu": B, "q_heads": hq, "kv_heads": hkv, "head_dim": d,
                 "window": wl.window, "context": int(ctx.max()) if wl.ctx_range is None else list(wl.ctx_range),
                 "layers": L, "attn_kernel": kernel, "parallelism": f"replicas x{world}",
-                "l2": f"inputs larger than L2: {L} layer pools, {layer_bytes / 2**20:.0f} MiB retained K/V each "
-                      f"({L * layer_bytes / 2**20:.0f} MiB per step vs 126 MiB L2)",
+                "l2": f"inputs larger than L2: {L} layer pools, {total_bytes / args.steps / 2**20:.0f} MiB "
+                      f"retained K/V read per step vs 126 MiB L2",
                 "step": ("per layer: dms_decode_step (append 1 token/seq + attention, one launch)" if fused else
-                         "per layer: dms_append (1 token/seq) + dms_decode_attention") + "; one dms_stats per step",
+                         "per layer: dms_append (1 token/seq) + dms_decode_attention") +
+                        ("; one dms_stats per layer per step" if depth else "; one dms_stats per step"),
             },
             "decode_steps_per_s_per_layer": n_layer_steps / (t_max_ms * 1e-3),
             "retained_bytes_per_step": total_bytes / args.steps,
             "compression_ratio": float(timed_tot[-1, 0] / timed_tot[-1, 1]),
+            **({"depth": {"cr_schedule": depth, "layer_cr": [
+                float(x) for x in per_layer[args.warmup + args.steps - 1, :, 0] /
+                per_layer[args.warmup + args.steps - 1, :, 1]]}} if depth else {}),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
                          "traffic": profile_traffic(wl.name, kernel,

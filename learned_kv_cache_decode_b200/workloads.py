@@ -20,6 +20,8 @@ from __future__ import annotations
 from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
+import dataclasses
+
 import numpy as np
 
 KV_CHUNK = 1024       # positions per independently seeded K/V block
@@ -84,6 +86,20 @@ WORKLOADS: dict[str, Workload] = {
     "longrun-2k-30k": Workload("longrun-2k-30k", 32, 28, 4, 128, "bf16", 256, 2048, None, 30000,
                                "bernoulli", (0.875,), 1005),
 }
+
+
+def depth_layers(wl: Workload, layers: int, cr_first: float, cr_last: float) -> list[Workload]:
+    """Per-layer workloads with compression that grows with depth ("Inference-Time
+    Hyper-Scaling with KV Cache Compression", paper summary, Method: early layers are
+    compressed less, Fig. 6). Layer l draws alpha ~ Bernoulli(p_l), with the long-context
+    ratio 1 / (1 - p_l) linear in l from cr_first to cr_last, each layer from its own
+    seed. Only alpha is drawn from a layer workload; K, V and queries come from `wl`."""
+    out = []
+    for l in range(layers):
+        cr = cr_first + (cr_last - cr_first) * (l / (layers - 1) if layers > 1 else 0.0)
+        out.append(dataclasses.replace(wl, name=f"{wl.name}-layer{l}", alpha_mode="bernoulli",
+                                       alpha_args=(1.0 - 1.0 / cr,), seed=wl.seed + 7919 * (l + 1)))
+    return out
 
 
 def _rng(*key: int) -> np.random.Generator:

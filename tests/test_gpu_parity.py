@@ -98,6 +98,41 @@ def test_stats_match_oracle_counts():
         run.close()
 
 
+def test_depth_wise_compression_per_layer():
+    """Layer caches whose compression grows with depth (W.depth_layers, CR 2 -> 16 over 4
+    layers) stepped through the fused path in turn: every output against the oracle, and
+    each layer's dms_stats (per-stream counts, per-head and overall CR) equal to the
+    oracle's counts; the measured ratios grow layer over layer."""
+    base = wl("depth", 3, 14, 2, 128, "bf16", 16, (300, 900), 6, 0.5, 43)
+    runs = [Run(x) for x in W.depth_layers(base, 4, 2.0, 16.0)]
+    try:
+        for run in runs:
+            run.prefill(chunk=257)
+        for step in range(base.decode_steps):
+            for run in runs:
+                out, Q = run.decode_step(step, fused=True)
+                torch.cuda.synchronize()
+                for b in range(base.batch):
+                    compare(out[b], run.oracle_out(b, Q[b]))
+        crs = []
+        for run in runs:
+            st = run.cache.stats()
+            o = run.sim.snapshot()
+            np.testing.assert_array_equal(st["retained"].cpu().numpy(), o["n"])
+            np.testing.assert_array_equal(st["seen"].cpu().numpy(), o["pos"])
+            tot = st["totals"].cpu().numpy()
+            assert tot[0] == o["pos"].sum() and tot[1] == o["n"].sum()
+            for h in range(base.num_kv_heads):
+                ref = o["pos"][h::base.num_kv_heads].sum() / o["n"][h::base.num_kv_heads].sum()
+                assert abs(float(st["head_cr"][h]) - ref) <= 1e-6 * ref
+            crs.append(tot[0] / tot[1])
+            assert run.cache.status() == _native.DMS_OK
+        assert crs == sorted(crs) and crs[-1] > 3 * crs[0], crs
+    finally:
+        for run in runs:
+            run.close()
+
+
 def test_empty_and_partial_batches():
     """Sequences never appended give zeros; decode over a subset, in any order."""
     case = wl("subset", 5, 8, 2, 64, "bf16", 16, (0, 300), 3, 0.5, 23)

@@ -56,3 +56,18 @@ def test_query_shapes():
         assert q.shape == (wl.batch, wl.num_q_heads, wl.head_dim)
         assert q.dtype == (np.uint16 if wl.dtype == "bf16" else np.float32)
         assert wl.num_q_heads % wl.num_kv_heads == 0
+
+
+def test_depth_layers_compress_more_with_depth():
+    """The per-layer schedule of depth-wise compression: alpha rates give long-context
+    ratios linear from the first to the last layer, each layer its own draws."""
+    base = W.WORKLOADS["qwen-r1-7b-32k"]
+    layers = W.depth_layers(base, 4, 2.0, 8.0)
+    assert [round(1.0 / (1.0 - x.alpha_args[0]), 9) for x in layers] == [2.0, 4.0, 6.0, 8.0]
+    assert len({x.seed for x in layers} | {base.seed}) == 5
+    rates = [float(W.alpha(x, 0, 0, 20000).mean()) for x in layers]
+    for x, r in zip(layers, rates):
+        assert abs(r - x.alpha_args[0]) < 0.01
+    assert rates == sorted(rates)
+    one = W.depth_layers(base, 1, 3.0, 9.0)
+    assert abs(1.0 / (1.0 - one[0].alpha_args[0]) - 3.0) < 1e-12
