@@ -305,6 +305,20 @@ dms_status dms_get_status(dms_cache* cache, cudaStream_t stream);
 /* Static description of a status code. */
 const char* dms_status_string(dms_status s);
 
+/* Failure-detection self-test (no counterpart in the paper): one block runs
+ * the library's two bounded waits on conditions that never come true.
+ *  1. a spin on a flag that nothing sets;
+ *  2. an mbarrier phase whose expected bytes never arrive (afterwards the
+ *     block completes that phase itself, so nothing is pending at exit).
+ * Each gives up after about 2^31 SM cycles (about a second), latches
+ * DMS_ERR_TIMEOUT into the cache's status word and returns. No fault, trap or
+ * hang. The cache is then poisoned as by any device error: dms_get_status
+ * returns DMS_ERR_TIMEOUT, and work-issuing calls are refused until
+ * dms_cache_reset.
+ *   timed_out  device int32 [2]: 1 where each wait gave up, else 0
+ * Async. */
+dms_status dms_selftest_bounded_waits(dms_cache* cache, cudaStream_t stream, int32_t* timed_out);
+
 /* Kernel launches issued by the library since the cache was created (host
  * counter, for accounting). */
 int64_t dms_launch_count(const dms_cache* cache);

@@ -173,6 +173,14 @@ class DmsCache:
                                              _ptr(K), _ptr(V)), "dms_gather_kv")
         return K, V
 
+    def selftest_bounded_waits(self) -> torch.Tensor:
+        """Run the library's bounded waits on conditions that never come true (about two
+        seconds). Each gives up and latches DMS_ERR_TIMEOUT, poisoning the cache until
+        reset(). Returns a device int32 [2]: 1 where each wait gave up."""
+        t = torch.zeros(2, dtype=torch.int32, device=self.device)
+        _native.check(self.lib.dms_selftest_bounded_waits(self._h, _stream(), _ptr(t)), "dms_selftest_bounded_waits")
+        return t
+
     def status(self) -> int:
         """Latched device status (syncs)."""
         return int(self.lib.dms_get_status(self._h, _stream()))

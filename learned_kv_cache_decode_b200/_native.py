@@ -30,7 +30,7 @@ DMS_ATTN_MMA = 2
 EXPORTS = ("dms_cache_create", "dms_cache_destroy", "dms_cache_reset", "dms_seq_reset", "dms_append",
            "dms_decode_attention", "dms_stats", "dms_snapshot", "dms_gather_kv", "dms_get_status",
            "dms_status_string", "dms_launch_count", "dms_decode_attention_noalloc", "dms_decode_step",
-           "dms_append_keyed", "dms_decode_step_keyed")
+           "dms_append_keyed", "dms_decode_step_keyed", "dms_selftest_bounded_waits")
 
 DMS_NOALLOC_MAX_STREAMS = 512
 DMS_NOALLOC_MAX_PIECES = 1024
@@ -106,6 +106,8 @@ def load() -> ctypes.CDLL:
     L.dms_gather_kv.restype = st
     L.dms_get_status.argtypes = [p, p]
     L.dms_get_status.restype = st
+    L.dms_selftest_bounded_waits.argtypes = [p, p, p]
+    L.dms_selftest_bounded_waits.restype = st
     L.dms_status_string.argtypes = [st]
     L.dms_status_string.restype = ctypes.c_char_p
     L.dms_launch_count.argtypes = [p]

@@ -10,6 +10,8 @@
 #include <new>
 #include <thread>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dms_internal.cuh"
 
 struct dms_cache {
@@ -38,6 +40,15 @@ struct dms_cache {
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range named after the API call, for profiler timelines (a no-op
+// unless a tool is attached).
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 // The cache whose kernels were launched last on each stream. Kernels that
 // write a cache are launched only through these calls, and each lets the next
@@ -137,6 +148,7 @@ cudaError_t alloc_next(const dms::Dev& dv, int grid, dms::NextPlan* np) {
 extern "C" {
 
 dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
+  const CallRange range("dms_cache_create");
   if (!cfg || !out) return DMS_ERR_INVALID;
   *out = nullptr;
   const dms_config& c = *cfg;
@@ -216,6 +228,7 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
 }
 
 dms_status dms_cache_destroy(dms_cache* h) {
+  const CallRange range("dms_cache_destroy");
   if (!h) return DMS_OK;
   int prev = -1;
   cudaGetDevice(&prev);
@@ -230,6 +243,7 @@ dms_status dms_cache_destroy(dms_cache* h) {
 }
 
 dms_status dms_cache_reset(dms_cache* h, cudaStream_t stream) {
+  const CallRange range("dms_cache_reset");
   if (!h) return DMS_ERR_INVALID;
   if (dms_status s = check_device(h)) return s;
   h->trust_tag = 0;
@@ -245,6 +259,7 @@ dms_status dms_cache_reset(dms_cache* h, cudaStream_t stream) {
 }
 
 dms_status dms_seq_reset(dms_cache* h, cudaStream_t stream, int32_t seq_id) {
+  const CallRange range("dms_seq_reset");
   if (!h || seq_id < 0 || seq_id >= h->cfg.max_seqs) return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
   h->launches += 1;
@@ -341,12 +356,14 @@ dms_status step_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const in
 dms_status dms_append(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                       const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
                       const uint8_t* alpha) {
+  const CallRange range("dms_append");
   return append_impl(h, stream, n_seqs, seq_ids, cu_tokens, total_tokens, K, V, alpha, -1);
 }
 
 dms_status dms_append_keyed(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                             const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
                             int32_t alpha_channel) {
+  const CallRange range("dms_append_keyed");
   if (alpha_channel < 0) return DMS_ERR_INVALID;
   return append_impl(h, stream, n_seqs, seq_ids, cu_tokens, total_tokens, K, V, nullptr, alpha_channel);
 }
@@ -354,6 +371,7 @@ dms_status dms_append_keyed(dms_cache* h, cudaStream_t stream, int32_t n_seqs, c
 dms_status dms_decode_attention(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                                 const void* Q, int32_t num_q_heads, float scale, void* out,
                                 dms_dtype out_dtype) {
+  const CallRange range("dms_decode_attention");
   if (!h || n_seqs < 0 || n_seqs > h->cfg.max_seqs) return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
   if (num_q_heads < h->cfg.num_kv_heads || num_q_heads % h->cfg.num_kv_heads != 0) return DMS_ERR_INVALID;
@@ -369,18 +387,21 @@ dms_status dms_decode_attention(dms_cache* h, cudaStream_t stream, int32_t n_seq
 dms_status dms_decode_step(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                            const void* K, const void* V, const uint8_t* alpha, const void* Q, int32_t num_q_heads,
                            float scale, void* out, dms_dtype out_dtype) {
+  const CallRange range("dms_decode_step");
   return step_impl(h, stream, n_seqs, seq_ids, K, V, alpha, -1, Q, num_q_heads, scale, out, out_dtype);
 }
 
 dms_status dms_decode_step_keyed(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                                  const void* K, const void* V, int32_t alpha_channel, const void* Q,
                                  int32_t num_q_heads, float scale, void* out, dms_dtype out_dtype) {
+  const CallRange range("dms_decode_step_keyed");
   if (alpha_channel < 0) return DMS_ERR_INVALID;
   return step_impl(h, stream, n_seqs, seq_ids, K, V, nullptr, alpha_channel, Q, num_q_heads, scale, out, out_dtype);
 }
 
 dms_status dms_stats(dms_cache* h, cudaStream_t stream, int32_t* retained, int32_t* seen, float* head_cr,
                      int64_t* totals) {
+  const CallRange range("dms_stats");
   if (!h) return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
   h->launches += 1;
@@ -391,6 +412,7 @@ dms_status dms_stats(dms_cache* h, cudaStream_t stream, int32_t* retained, int32
 
 dms_status dms_snapshot(dms_cache* h, cudaStream_t stream, int32_t* page_table, int32_t* n_pages, int32_t* n,
                         int32_t* pos, int32_t* slot_pos, int32_t* free_list, int32_t* free_count) {
+  const CallRange range("dms_snapshot");
   if (!h) return DMS_ERR_INVALID;
   if (dms_status s = check_device(h)) return s;
   const dms::Dev& dv = h->dv;
@@ -412,6 +434,7 @@ dms_status dms_snapshot(dms_cache* h, cudaStream_t stream, int32_t* page_table, 
 
 dms_status dms_gather_kv(dms_cache* h, cudaStream_t stream, int32_t seq_id, int32_t kv_head, int32_t rows_cap,
                          void* K_out, void* V_out) {
+  const CallRange range("dms_gather_kv");
   if (!h || seq_id < 0 || seq_id >= h->cfg.max_seqs || kv_head < 0 || kv_head >= h->cfg.num_kv_heads)
     return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
@@ -423,6 +446,7 @@ dms_status dms_gather_kv(dms_cache* h, cudaStream_t stream, int32_t seq_id, int3
 }
 
 dms_status dms_get_status(dms_cache* h, cudaStream_t stream) {
+  const CallRange range("dms_get_status");
   if (!h) return DMS_ERR_INVALID;
   if (dms_status s = check_device(h)) return s;
   int32_t word = 0;
@@ -449,5 +473,14 @@ const char* dms_status_string(dms_status s) {
 }
 
 int64_t dms_launch_count(const dms_cache* h) { return h ? h->launches : 0; }
+
+dms_status dms_selftest_bounded_waits(dms_cache* h, cudaStream_t stream, int32_t* timed_out) {
+  const CallRange range("dms_selftest_bounded_waits");
+  if (!h || !timed_out) return DMS_ERR_INVALID;
+  if (dms_status s = check_device(h)) return s;
+  h->launches += 1;
+  note_launch(h, h->device, stream);   // it writes the cache's status word
+  return from_cuda(dms::launch_bounded_wait_selftest(h->dv, stream, timed_out));
+}
 
 }  // extern "C"

@@ -474,6 +474,34 @@ cudaError_t prepare_aux_kernels() {
   return cudaSuccess;
 }
 
+// Failure-detection self-test: the library's two bounded waits, on conditions
+// that never come true, in one thread. Each gives up after about 2^31 SM
+// cycles, latches DMS_ERR_TIMEOUT and returns; the mbarrier's pending phase is
+// then completed by the thread itself, so nothing is left pending at exit.
+__global__ void __launch_bounds__(32) bounded_wait_selftest_kernel(int32_t* ctrl, int32_t* timed_out) {
+  __shared__ int never;        // a flag nothing sets
+  __shared__ int abort_flag;
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  never = 0;
+  abort_flag = 0;
+  wait_flag_ge(&never, 1, &abort_flag, ctrl);   // raises abort_flag when it gives up
+  timed_out[0] = abort_flag != 0;
+  abort_flag = 0;
+  const uint32_t b = smem_addr(&bar);
+  mbar_init(b, 1);
+  fence_mbar_init();
+  mbar_arrive_expect_tx(b, 16);   // 16 bytes that no copy will bring
+  timed_out[1] = mbar_wait_bounded(b, 0, &abort_flag, ctrl) ? 0 : 1;
+  mbar_complete_tx(b, 16);        // close the phase
+  mbar_wait_timed(b, 0, ctrl);
+}
+
+cudaError_t launch_bounded_wait_selftest(const Dev& dv, cudaStream_t st, int32_t* timed_out) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(dv.ctrl, timed_out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_init_state(const Dev& dv, cudaStream_t st) {
   init_state_kernel<<<256, 256, 0, st>>>(dv);
   return cudaGetLastError();

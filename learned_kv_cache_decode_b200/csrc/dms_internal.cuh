@@ -113,6 +113,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
+// Complete `bytes` of the current phase's expected transactions from a thread.
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -368,6 +372,7 @@ cudaError_t launch_append_bulk(const Dev& dv, cudaStream_t st, int n_seqs, const
                                const int32_t* cu_tokens, int total_tokens, const void* K, const void* V,
                                const uint8_t* alpha, int alpha_channel, int* launches);
 cudaError_t launch_reset_seq(const Dev& dv, cudaStream_t st, int seq);
+cudaError_t launch_bounded_wait_selftest(const Dev& dv, cudaStream_t st, int32_t* timed_out);
 cudaError_t launch_stats(const Dev& dv, cudaStream_t st, int32_t* retained, int32_t* seen, float* head_cr,
                          int64_t* totals);
 cudaError_t launch_gather(const Dev& dv, cudaStream_t st, int seq, int kvh, int rows_cap, void* Kout,

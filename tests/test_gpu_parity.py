@@ -581,6 +581,46 @@ def test_attention_of_two_caches_captured_in_a_graph_between_eager_calls():
             run.close()
 
 
+def test_bounded_waits_give_up_latch_timeout_and_reset_recovers():
+    """Failure detection without a GPU fault. The library's two bounded waits run on
+    conditions that never come true: a flag nothing sets, and an mbarrier phase whose
+    bytes never arrive. Each gives up after about a second and latches DMS_ERR_TIMEOUT.
+    The cache is then poisoned; dms_cache_reset brings it back, and the same cache (and
+    context) decodes correctly again."""
+    import oracle
+    case = wl("selftest", 2, 8, 2, 64, "bf16", 16, (20, 300), 3, 0.5, 44)
+    run = Run(case)
+    try:
+        run.prefill(chunk=64)
+        t = run.cache.selftest_bounded_waits()
+        torch.cuda.synchronize()
+        assert t.cpu().tolist() == [1, 1]
+        assert run.cache.status() == _native.DMS_ERR_TIMEOUT
+        with pytest.raises(_native.DmsError) as err:
+            run.cache.decode_attention(torch.tensor([0], dtype=torch.int32, device="cuda"),
+                                       torch.zeros((1, 8, 64), dtype=torch.bfloat16, device="cuda"))
+        assert err.value.code == _native.DMS_ERR_POISONED
+        run.cache.reset()
+        assert run.cache.status() == _native.DMS_OK
+        # a fresh start on the same cache, checked against a fresh oracle simulator
+        cfg = run.cache.cfg
+        run.sim.close()
+        run.sim = oracle.Sim(case.batch, case.num_kv_heads, case.window, cfg.max_pages, cfg.max_pages_per_stream)
+        run.seen[:] = 0
+        run._blk.clear()
+        run.prefill(chunk=64)
+        run.check_metadata()
+        for step in range(case.decode_steps):
+            out, Q = run.decode_step(step, fused=True)
+            torch.cuda.synchronize()
+            for b in range(case.batch):
+                compare(out[b], run.oracle_out(b, Q[b]))
+        run.check_metadata()
+        assert run.cache.status() == _native.DMS_OK
+    finally:
+        run.close()
+
+
 # ---------------------------------------------------------------------------
 # alpha read from a designated key channel (dms_append_keyed, dms_decode_step_keyed)
 
