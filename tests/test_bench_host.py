@@ -74,3 +74,36 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
     j = json.loads(lines[0])
     assert j["impl"] == "reference" and j["unit"] == "GB/s" and j["value"] > 0
     assert j["cpu_baseline"]["kind"] == "oracle" and j["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_code_fingerprint_ignores_comments_only(tmp_path):
+    """The profile summaries are matched to the kernel by a hash of its code with comments
+    and whitespace removed: a comment edit keeps the match, a code edit breaks it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = tmp_path / "a.cu"
+    a.write_text("// header\nint f(int x) {  /* a\n block */ return x + 1; }  // tail\n")
+    b = tmp_path / "b.cu"
+    b.write_text("// another header\n\nint f(int x) {\n  return x + 1;\n}\n")
+    c = tmp_path / "c.cu"
+    c.write_text("int f(int x) { return x + 2; }\n")
+    assert bench.code_fingerprint(str(a)) == bench.code_fingerprint(str(b))
+    assert bench.code_fingerprint(str(a)) != bench.code_fingerprint(str(c))
+
+
+def test_profile_traffic_needs_the_matching_code_hash():
+    """bench.py reports `traffic` from a committed profile summary only while its recorded
+    code hash matches the kernel source."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import re as _re
+    src = os.path.join(ROOT, "learned_kv_cache_decode_b200", "csrc", "dms_attention.cu")
+    path = os.path.join(ROOT, "profiles", "dms_decode_step_mma_qwen-r1-7b-32k.md")
+    text = open(path).read()
+    recorded = _re.search(r"code_sha256:\s*([0-9a-f]{64})", text).group(1)
+    traffic = bench.profile_traffic("qwen-r1-7b-32k", "mma", "dms_decode_step")
+    if recorded == bench.code_fingerprint(src):
+        assert traffic is not None and traffic > 1e8
+    else:
+        assert traffic is None
+    assert bench.profile_traffic("no-such-workload", "mma", "dms_decode_step") is None
