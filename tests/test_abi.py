@@ -75,3 +75,29 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "_lib", None)
     with pytest.raises(ImportError):
         _native.load()
+
+
+def test_a_c_program_compiles_against_the_header_links_and_calls_the_library(lib, tmp_path):
+    """The boundary is plain C: dms.h compiles as strict C11, and a C program links
+    against libdms.so and calls it (a host-only call: there is no GPU here)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_dms.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <string.h>\n#include "dms.h"\n'
+        "int main(void) {\n"
+        '  if (strcmp(dms_status_string(DMS_OK), "ok") != 0) return 1;\n'
+        "  if (dms_launch_count(NULL) != 0) return 2;\n"
+        "  if (dms_cache_destroy(NULL) != DMS_OK) return 3;\n"
+        '  printf("%s\\n", dms_status_string(DMS_ERR_TIMEOUT));\n'
+        "  return 0;\n}\n")
+    pkg = os.path.join(ROOT, "learned_kv_cache_decode_b200")
+    exe = tmp_path / "use_dms"
+    cuda_inc = "/usr/local/cuda/include"
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", cuda_inc, str(src), "-o", str(exe), "-L", pkg, "-ldms", f"-Wl,-rpath,{pkg}"],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True)
+    assert out.stdout.strip() == "bounded wait timed out inside a kernel"
