@@ -419,6 +419,30 @@ def test_window_sweep(w, fused):
         run.close()
 
 
+@pytest.mark.parametrize("batch", [256, 257], ids=["1024_streams_fused", "1028_streams_two_launches"])
+def test_decode_step_at_the_stream_limit_and_past_it(batch):
+    """dms_decode_step at the fused kernel's limit of 1024 streams (256 sequences x 4 KV
+    heads) and just past it, where the call issues the two launches instead: metadata bit
+    for bit and every sequence's output against the oracle at every step."""
+    case = wl(f"limit-{batch}", batch, 8, 4, 64, "bf16", 8, (10, 60), 3, 0.6, 45)
+    run = Run(case)
+    try:
+        run.prefill(chunk=64)
+        run.check_metadata()
+        for step in range(case.decode_steps):
+            before = run.cache.launches()
+            out, Q = run.decode_step(step, fused=True)
+            launched = run.cache.launches() - before
+            assert launched == 1 if batch * case.num_kv_heads <= 1024 else launched >= 2, launched
+            torch.cuda.synchronize()
+            for b in range(batch):
+                compare(out[b], run.oracle_out(b, Q[b]))
+            run.check_metadata()
+        assert run.cache.status() == _native.DMS_OK
+    finally:
+        run.close()
+
+
 def test_fused_step_after_another_caches_stats_kernel():
     """Fused steps on cache A with a dms_stats call on cache B between them. The stats
     kernel lets the next kernel start at once, so A's previous step may still be running
