@@ -84,14 +84,33 @@ def alpha_from_keys(K: np.ndarray, channel: int) -> np.ndarray:
     """Eviction decisions read from a designated key channel: uint8 [..., Hkv].
 
     Method section of the paper summary: one neuron of the K projection per head
-    is repurposed to produce the eviction logit. At inference (reading R4) the
-    token is marked iff that logit is > 0; zero and NaN keep it. K holds stored
+    is repurposed to produce the eviction logit. At inference the token is
+    marked iff that logit is > 0 (the plainest binarisation of the logit; the
+    pages do not state one); zero and NaN keep it. K holds stored
     values: bf16 bits as uint16, or float32.
     """
     x = np.asarray(K)
     logit = (x[..., channel].astype(np.uint32) << np.uint32(16)).view(np.float32) if x.dtype == np.uint16 \
         else x[..., channel].astype(np.float32)
     return (logit > 0).astype(np.uint8)
+
+
+def alpha_from_queries(Q: np.ndarray, num_kv_heads: int, head: int, channel: int) -> np.ndarray:
+    """Eviction decisions read from a designated channel of one query head per KV
+    head: uint8 [..., Hkv].
+
+    Method section of the paper summary: the eviction logit may come from a
+    neuron of the Q projection instead of the K one. The decision stays one per
+    KV head, so one query head of each group is designated: query heads
+    k*g .. k*g+g-1 belong to KV head k (contiguous GQA grouping) and ``head``
+    picks k*g + head. The sign rule is that of alpha_from_keys. Q holds stored
+    values [..., Hq, d]: bf16 bits as uint16, or float32.
+    """
+    x = np.asarray(Q)
+    g = x.shape[-2] // num_kv_heads
+    assert 0 <= head < g and g * num_kv_heads == x.shape[-2]
+    rows = x[..., [k * g + head for k in range(num_kv_heads)], :]   # [..., Hkv, d]
+    return alpha_from_keys(rows, channel)
 
 
 def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, alpha_seq: np.ndarray,
@@ -232,5 +251,6 @@ def available() -> bool:
         return False
 
 
-__all__ = ["lib", "visible_positions", "retained_count_closed_form", "attention", "decode_gqa",
+__all__ = ["lib", "visible_positions", "retained_count_closed_form", "alpha_from_keys", "alpha_from_queries",
+           "attention", "decode_gqa",
            "attention_batch", "Sim", "available"]

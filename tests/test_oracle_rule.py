@@ -247,3 +247,50 @@ def test_alpha_from_keys_reads_only_the_designated_channel():
         K3 = K.copy()
         K3[..., c] *= -1.0   # flipping the logit flips every non-zero decision
         np.testing.assert_array_equal(oracle.alpha_from_keys(K3, c), 1 - a)
+
+
+def _golden_queries():
+    q, picks = [], []
+    for line in open(os.path.join(GOLD, "alpha_from_queries.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        key, *rest = line.split()
+        if key == "q":
+            q.append([float(x) for x in rest[1:]])
+        elif key == "pick":
+            picks.append((int(rest[0]), int(rest[1]), [int(rest[2]), int(rest[3])]))
+    return np.array(q, dtype=np.float32), picks
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_golden_alpha_from_queries(dtype):
+    """The hand-worked picks fix which query head of each group holds the logit
+    (contiguous grouping: an interleaved one gives different bits for some picks)."""
+    q, picks = _golden_queries()
+    assert q.shape == (6, 4) and len(picks) >= 8
+    Q = q[None]                                           # one token [1, Hq, d]
+    if dtype == "bf16":
+        Q = (Q.view(np.uint32) >> np.uint32(16)).astype(np.uint16)   # exact: every value fits bf16
+    for head, ch, want in picks:
+        a = oracle.alpha_from_queries(Q, 2, head, ch)
+        assert a.shape == (1, 2) and a.dtype == np.uint8
+        assert a[0].tolist() == want, (head, ch, a[0].tolist(), want)
+
+
+def test_alpha_from_queries_is_the_key_rule_on_the_designated_heads():
+    """With g = 1 the query rule is the key rule; with g > 1 it reads only the
+    designated head of each group, whatever the other heads hold."""
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((40, 4, 16)).astype(np.float32)
+    np.testing.assert_array_equal(oracle.alpha_from_queries(X, 4, 0, 9), oracle.alpha_from_keys(X, 9))
+    Q = rng.standard_normal((40, 12, 16)).astype(np.float32)   # Hkv = 3, g = 4
+    a = oracle.alpha_from_queries(Q, 3, 2, 5)
+    Q2 = Q.copy()
+    for k in range(3):
+        for j in (0, 1, 3):
+            Q2[:, 4 * k + j] = -Q2[:, 4 * k + j]   # the other heads of each group do not matter
+    np.testing.assert_array_equal(oracle.alpha_from_queries(Q2, 3, 2, 5), a)
+    Q3 = Q.copy()
+    Q3[:, [2, 6, 10], 5] *= -1.0                   # flipping the designated logits flips every decision
+    np.testing.assert_array_equal(oracle.alpha_from_queries(Q3, 3, 2, 5), 1 - a)
