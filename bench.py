@@ -59,6 +59,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--per-workload", dest="per_workload", action="store_true", default=True,
+                    help="also measure the other workloads (and a dense run) into a per_workload block (default)")
+    ap.add_argument("--no-per-workload", dest="per_workload", action="store_false")
     ap.add_argument("--depth", default="",
                     help="CR_FIRST,CR_LAST: compression growing with depth, each layer cache with its "
                          "own alpha rate (workloads.depth_layers); per-layer dms_stats at every step; "
@@ -299,29 +302,41 @@ def run_reference(args, wl, world, rank):
 # ---------------------------------------------------------------------------
 # our arm
 
-def main():
-    args = parse_args()
-    wl = W.WORKLOADS[args.workload]
-    if args.window:
-        import dataclasses
-        wl = dataclasses.replace(wl, window=args.window)
-    depth = [float(x) for x in args.depth.split(",")] if args.depth else None
-    if depth:
-        args.no_e2e = True   # the e2e pass copies one alpha row per step for all layers
-    world, rank, local = dist_setup(args)
-    if args.impl == "reference":
-        run_reference(args, wl, world, rank)
-        return
+NOMINAL_HBM_GBS = 8000.0   # the B200's nominal HBM3e bandwidth (about 8 TB/s), for the second fraction
 
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def time_oracle_one_core(items, window, scale, target_s):
+    """The oracle's single-stream routine called stream after stream (one core)."""
+    import oracle
+    reps, t_total = 0, 0.0
+    while t_total < target_s or reps == 0:
+        t0 = time.perf_counter()
+        for q, K, V, a in items:
+            oracle.attention(q, K, V, a, window, scale)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    return reps, t_total
+
+
+def measure(wl, args, world, rank, local, dev, *, steps, warmup, layers=0, depth=None, want_e2e=True,
+            want_cpu=False, fused=True):
+    """Prefill L layer caches of workload `wl`, then time decode steps. Returns the
+    figures of one workload (and, with want_e2e / want_cpu, its e2e and CPU passes)."""
     import torch
     import torch.distributed as dist
     from learned_kv_cache_decode_b200 import DmsCache
-
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     # this rank's sequences (weak scaling: every rank runs a full batch of its own sequences)
     seqs = rank_sequences(rank, wl.batch)
@@ -331,7 +346,7 @@ def main():
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     burst_steps = 5
     # timed, per-launch, burst and e2e passes
-    n_dec = args.warmup + args.steps * (2 if args.no_e2e else 3) + burst_steps
+    n_dec = warmup + steps * (3 if want_e2e else 2) + burst_steps
     mps = int((ctx.max() + n_dec) // 16 + 2)
     scale = 1.0 / math.sqrt(d)
 
@@ -347,12 +362,13 @@ def main():
         c.append(ids, dK, dV, alpha, cu_tokens=d_cu)
         return c
 
+    A_first = None
     if depth:
         # One alpha stream per layer (compression growing with depth); worst-case pools.
-        L = args.layers or 8
+        L = layers or 8
         layer_wls = W.depth_layers(wl, L, depth[0], depth[-1])
         pool = B * hkv * mps
-        caches, A_first = [], None
+        caches = []
         for lw in layer_wls:
             a_l = np.concatenate([W.alpha(lw, b, 0, int(c_)) for b, c_ in zip(seqs, ctx)])
             A_first = a_l if A_first is None else A_first
@@ -369,7 +385,7 @@ def main():
         del probe
         pool = int(((retained + 15) // 16).sum()) + B * hkv * (n_dec // 16 + 2)
         layer_bytes = retained0 * d * 2 * wl.elem_bytes
-        L = args.layers or max(1, min(32, math.ceil(8 * L2_BYTES / max(layer_bytes, 1))))
+        L = layers or max(1, min(32, math.ceil(8 * L2_BYTES / max(layer_bytes, 1))))
         caches = [new_layer(pool, dA) for _ in range(L)]
     torch.cuda.synchronize()
     del dK, dV, dA
@@ -398,12 +414,9 @@ def main():
     pK, pV, pA, pQ = t_K.data_ptr(), t_V.data_ptr(), t_A.data_ptr(), t_Q.data_ptr()
     pT = totals.data_ptr()
     pids = ids.data_ptr()
-    launches0 = sum(c.launches() for c in caches)
     ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps * L)]
-    t_pl = args.warmup + args.steps   # first step of the per-launch pass
-
-    fused = args.step == "fused"
+                for _ in range(steps * L)]
+    t_pl = warmup + steps   # first step of the per-launch pass
     odt = 0 if tdt == torch.bfloat16 else 1
 
     def alpha_ptr(t, l):
@@ -432,15 +445,16 @@ def main():
             if rc:
                 raise RuntimeError(f"library call failed ({rc})")
 
-    for t in range(args.warmup):
+    for t in range(warmup):
         step(t, False)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    launches0 = sum(c.launches() for c in caches)
     ev_start, ev_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         ev_start.record(stream)
-        for t in range(args.warmup, args.warmup + args.steps):
+        for t in range(warmup, warmup + steps):
             step(t, False)
         ev_end.record(stream)
         torch.cuda.synchronize()
@@ -453,19 +467,19 @@ def main():
     # every attention launch. The events serialise each launch behind the one
     # before it, so these durations include the launch latency that the
     # timed region overlaps; they are the conservative per-kernel figure.
-    for t in range(t_pl, t_pl + args.steps):
+    for t in range(t_pl, t_pl + steps):
         step(t, True)
     torch.cuda.synchronize()
     tot = totals.cpu().numpy()                                         # [steps, 1 or L, 2]
     per_layer = tot if depth else np.repeat(tot, L, axis=1)            # [steps, L, 2]
-    timed_tot = per_layer[args.warmup:args.warmup + args.steps].sum(axis=1)   # [steps, 2] over layers
-    bytes_launch = per_layer[args.warmup:args.warmup + args.steps, :, 1].astype(np.float64) * d * 2 * wl.elem_bytes
+    timed_tot = per_layer[warmup:warmup + steps].sum(axis=1)           # [steps, 2] over layers
+    bytes_launch = per_layer[warmup:warmup + steps, :, 1].astype(np.float64) * d * 2 * wl.elem_bytes
     total_bytes = float(bytes_launch.sum())
     same = [c.stats()["totals"].cpu().numpy().tolist() for c in caches]
     if not depth and any(x != same[0] for x in same):
         raise RuntimeError(f"layer caches diverged: {same}")
     attn_ms = np.array([a.elapsed_time(b) for a, b in ev_pairs])
-    bytes_pl = per_layer[t_pl:t_pl + args.steps, :, 1].astype(np.float64) * d * 2 * wl.elem_bytes
+    bytes_pl = per_layer[t_pl:t_pl + steps, :, 1].astype(np.float64) * d * 2 * wl.elem_bytes
     status = [c.status() for c in caches]
     if any(status):
         raise RuntimeError(f"device status {status}")
@@ -473,14 +487,13 @@ def main():
     # max over ranks of the timed region; whole-job bytes
     t_max_ms, bytes_all = reduce_over_ranks(t_ms, total_bytes, world, dev)
     value = bytes_all / (t_max_ms * 1e-3) / 1e9
-
     achieved_iso = float(bytes_pl.mean()) / (float(attn_ms.mean()) * 1e-3) / 1e9
 
     # Burst: `burst_steps` more steps between one event pair, no event between
     # launches, so each launch's set-up overlaps the launch before it
     # (programmatic dependent launch). Separate mode times the attention
     # launches alone. Reported beside the per-launch figure, not instead of it.
-    t_b = t_pl + args.steps
+    t_b = t_pl + steps
     e_b0, e_b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if fused:
         e_b0.record(stream)
@@ -510,30 +523,38 @@ def main():
     # it: an event between two launches makes each start only once the one
     # before has finished, which removes the overlap of consecutive launches.
     if fused:
-        launch_ms = t_ms / (args.steps * L)
+        launch_ms = t_ms / (steps * L)
         achieved = float(bytes_launch.mean()) / (launch_ms * 1e-3) / 1e9
-        launch_timing = ("timed region (CUDA events at its two ends) over its step launches; "
-                         "isolated: an event pair around every launch, in a second pass over the next steps")
     else:
         launch_ms = burst_ms
         achieved = achieved_burst
-        launch_timing = ("attention launches back to back between one event pair (the burst); "
-                         "isolated: an event pair around every launch, in a second pass over the next steps")
     peak, peak_kind = peaks()
-    kernel = {"auto": "mma" if tdt == torch.bfloat16 else "simt"}.get(args.attn_kernel, args.attn_kernel)
+
+    res = {
+        "wl": wl, "L": L, "B": B, "hq": hq, "hkv": hkv, "d": d, "ctx": ctx, "value": value, "t_max_ms": t_max_ms,
+        "steps": steps, "total_bytes": total_bytes, "launches": launches, "clocks": clk.summary(),
+        "timed_tot": timed_tot, "per_layer": per_layer, "warmup": warmup,
+        "bytes_launch": float(bytes_launch.mean()) if fused else float(bytes_pl.mean()),
+        "launch_ms": launch_ms, "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+        "attn_ms": attn_ms, "achieved_iso": achieved_iso, "burst_ms": burst_ms, "achieved_burst": achieved_burst,
+    }
 
     # ---- end-to-end pass through the public API with pinned host buffers. Per
-    # step: one host-to-device copy of each input (every layer appends the same
-    # new token rows) and one device-to-host copy of every layer's output. The
-    # copies run on their own stream, double-buffered, so step t+1's inputs and
-    # step t-1's outputs move while step t computes; events order every reuse.
-    e2e = None
-    if not args.no_e2e:
-        hK, hV, hA, hQ = (to_torch(x, None).pin_memory() for x in (Kd, Vd, Ad, Qd))
+    # step and per layer: one host-to-device copy of each input a model step
+    # feeds that layer (its new K and V rows, alpha and Q; every layer gets its
+    # own copy of the bytes) and one device-to-host copy of every layer's
+    # output. The copies run on their own stream, double-buffered, so step
+    # t+1's inputs and step t-1's outputs move while step t computes; events
+    # order every reuse.
+    if want_e2e and not depth:
+        rep = lambda x: np.ascontiguousarray(np.broadcast_to(x[:, None], (x.shape[0], L) + x.shape[1:]))
+        hK, hV, hA, hQ = (to_torch(rep(x), None).pin_memory() for x in (Kd, Vd, Ad, Qd))   # [steps, L, ...]
         h_out = [torch.empty((L, B, hq, d), dtype=tdt).pin_memory() for _ in range(2)]
         d_out = [torch.empty((L, B, hq, d), dtype=tdt, device=dev) for _ in range(2)]
-        stage = [(torch.empty((B, hkv, d), dtype=tdt, device=dev), torch.empty((B, hkv, d), dtype=tdt, device=dev),
-                  torch.empty((B, hkv), dtype=torch.uint8, device=dev), torch.empty((B, hq, d), dtype=tdt, device=dev))
+        stage = [(torch.empty((L, B, hkv, d), dtype=tdt, device=dev),
+                  torch.empty((L, B, hkv, d), dtype=tdt, device=dev),
+                  torch.empty((L, B, hkv), dtype=torch.uint8, device=dev),
+                  torch.empty((L, B, hq, d), dtype=tdt, device=dev))
                  for _ in range(2)]
         copy_s = torch.cuda.Stream(device=dev)
         ev = lambda: torch.cuda.Event()
@@ -559,20 +580,20 @@ def main():
         e_a.record(stream)
         copy_s.wait_stream(stream)
         h2d(t0_e2e)
-        for t in range(t0_e2e, t0_e2e + args.steps):
+        for t in range(t0_e2e, t0_e2e + steps):
             p = t % 2
             k_, v_, a_, q_ = stage[p]
-            if t + 1 < t0_e2e + args.steps:
+            if t + 1 < t0_e2e + steps:
                 h2d(t + 1)
             stream.wait_event(h2d_done[p])
             if t - 2 >= t0_e2e:
                 stream.wait_event(d2h_done[p])    # step t-2's outputs have left this buffer
             for l in range(L):
                 if fused:
-                    caches[l].decode_step(ids, k_, v_, a_, q_, scale=scale, out=d_out[p][l])
+                    caches[l].decode_step(ids, k_[l], v_[l], a_[l], q_[l], scale=scale, out=d_out[p][l])
                 else:
-                    caches[l].append(ids, k_, v_, a_)
-                    caches[l].decode_attention(ids, q_, scale=scale, out=d_out[p][l])
+                    caches[l].append(ids, k_[l], v_[l], a_[l])
+                    caches[l].decode_attention(ids, q_[l], scale=scale, out=d_out[p][l])
                 if l == 0:
                     lib.dms_stats(hs[l], sp, None, None, None, pT + t * 16)
             comp_done[p].record(stream)
@@ -584,76 +605,185 @@ def main():
         e_b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e_a.elapsed_time(e_b)
-        tot2 = totals.cpu().numpy()[t0_e2e:t0_e2e + args.steps, 0]   # layer 0 stands for all (no --depth)
+        tot2 = totals.cpu().numpy()[t0_e2e:t0_e2e + steps, 0]   # layer 0 stands for all (no --depth)
         e2e_bytes = float(tot2[:, 1].astype(np.float64).sum()) * L * d * 2 * wl.elem_bytes
         e2e_ms, e2e_bytes = reduce_over_ranks(e2e_ms, e2e_bytes, world, dev)
-        h2d_b = 2 * row_kv + B * hkv + row_q
+        h2d_b = L * (2 * row_kv + B * hkv + row_q)
         d2h_b = L * B * hq * d * wl.elem_bytes
-        e2e = {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d_b,
-               "d2h_bytes_per_step": d2h_b, "ms_per_step": e2e_ms / args.steps,
-               "copies": "own stream, double-buffered (step t+1 in, step t-1 out while step t computes)"}
+        res["e2e"] = {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d_b,
+                      "d2h_bytes_per_step": d2h_b, "ms_per_step": e2e_ms / steps,
+                      "copies": "per layer: new K, V rows, alpha and Q in, output out; own stream, "
+                                "double-buffered (step t+1 in, step t-1 out while step t computes)"}
 
     # ---- CPU baseline: the oracle on a bounded sample of the same step (rank 0, N = 1)
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if want_cpu:
         sample_seqs = list(range(min(B, 2)))
         A_s, Ad_s = (A_first, Ad[0]) if depth else (A_p, Ad)   # --depth: layer 0's decisions
-        items, nbytes = oracle_sample(wl, [seqs[i] for i in sample_seqs], args.warmup + args.steps,
+        items, nbytes = oracle_sample(wl, [seqs[i] for i in sample_seqs], warmup + steps,
                                       (K_p, V_p, A_s, offs),
                                       (Kd[:, sample_seqs], Vd[:, sample_seqs], Ad_s[:, sample_seqs],
                                        Qd[:, sample_seqs]))
         reps, t_cpu, threads = time_oracle(items, wl.window, scale, args.cpu_seconds)
-        cpu = {"value": nbytes * reps / t_cpu / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": f"{len(items)} streams (sequences {sample_seqs}, every KV head) at the last timed step, "
-                         f"repeated {reps}x ({t_cpu:.1f} s); fp64 definition-form oracle, OpenMP over streams"}
+        reps1, t_cpu1 = time_oracle_one_core(items, wl.window, scale, args.cpu_seconds / 2)
+        # per decode step of the whole workload (every stream of every layer), from the sample's rate
+        step_bytes = total_bytes / steps
+        res["cpu"] = {
+            "value": nbytes * reps / t_cpu / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+            "one_core": {"value": nbytes * reps1 / t_cpu1 / 1e9, "unit": "GB/s", "cores": 1,
+                         "ms_per_step": step_bytes / (nbytes * reps1 / t_cpu1) * 1e3},
+            "ms_per_step": step_bytes / (nbytes * reps / t_cpu) * 1e3,
+            "sample": f"{len(items)} streams (sequences {sample_seqs}, every KV head) at the last timed step, "
+                      f"repeated {reps}x on {threads} threads ({t_cpu:.1f} s) and {reps1}x on one core "
+                      f"({t_cpu1:.1f} s); fp64 definition-form oracle; ms_per_step scales the sample's rate "
+                      f"to every stream of every layer of one step"}
+
+    for c in caches:
+        c.close()
+    del caches
+    torch.cuda.empty_cache()
+    return res
+
+
+def brief(res):
+    """The per-workload figures of one measurement."""
+    wl = res["wl"]
+    peak = res["peak"]
+    return {
+        "value": res["value"], "unit": "GB/s", "ms_per_step": res["t_max_ms"] / res["steps"],
+        "layers": res["L"], "steps": res["steps"],
+        "bytes_per_launch": res["bytes_launch"], "launch_ms": res["launch_ms"],
+        "frac": res["achieved"] / peak, "frac_nominal": res["achieved"] / NOMINAL_HBM_GBS,
+        "launch_ms_isolated": float(res["attn_ms"].mean()),
+        "frac_isolated": res["achieved_iso"] / peak, "frac_isolated_nominal": res["achieved_iso"] / NOMINAL_HBM_GBS,
+        "compression_ratio": float(res["timed_tot"][-1, 0] / res["timed_tot"][-1, 1]),
+        "decode_steps_per_s_per_layer": res["steps"] * res["L"] / (res["t_max_ms"] * 1e-3),
+        "context": int(res["ctx"].max()) if wl.ctx_range is None else list(wl.ctx_range),
+        "clocks_sm_mhz": res["clocks"].get("sm_mhz"),
+    }
+
+
+def per_workload_runs(args, world, rank, local, dev, main_wl):
+    """The other workloads, each measured with fewer steps, no e2e and no CPU pass;
+    the long run at both ends of its decode loop; a dense (all kept) run of the
+    32K workload for context; the tiny workload as a correctness-only note."""
+    import dataclasses
+    steps = min(args.steps, 20)
+    runs = {}
+    lr = W.WORKLOADS["longrun-2k-30k"]
+    jobs = [
+        ("llama3.2-1b", W.WORKLOADS["llama3.2-1b"]),
+        ("qwen-r1-32b-chains", W.WORKLOADS["qwen-r1-32b-chains"]),
+        ("longrun-2k-30k@2k", lr),
+        # the state after its 30K decode steps: the prompt and every decode token appended at
+        # once (a bulk append equals token-by-token appends), then timed
+        ("longrun-2k-30k@32k", dataclasses.replace(lr, context=lr.context + lr.decode_steps)),
+        ("qwen-r1-7b-32k-dense", dataclasses.replace(W.WORKLOADS["qwen-r1-7b-32k"], alpha_mode="bernoulli",
+                                                     alpha_args=(0.0,))),
+    ]
+    if main_wl.name != "qwen-r1-7b-32k":
+        jobs.insert(0, ("qwen-r1-7b-32k", W.WORKLOADS["qwen-r1-7b-32k"]))
+    for name, wl in jobs:
+        if wl.name == main_wl.name and wl == main_wl:
+            continue
+        t0 = time.perf_counter()
+        r = measure(wl, args, world, rank, local, dev, steps=steps, warmup=3, want_e2e=False, want_cpu=False,
+                    fused=args.step == "fused")
+        runs[name] = brief(r)
+        runs[name]["wall_s"] = time.perf_counter() - t0
+    runs["tiny"] = {"note": "correctness only: one fp32 stream of about 280 retained tokens (0.15 MB per step), "
+                            "checked every step against the oracle in tests/test_gpu_configs.py"}
+    return runs
+
+
+def main():
+    args = parse_args()
+    wl = W.WORKLOADS[args.workload]
+    if args.window:
+        import dataclasses
+        wl = dataclasses.replace(wl, window=args.window)
+    depth = [float(x) for x in args.depth.split(",")] if args.depth else None
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    fused = args.step == "fused"
+    res = measure(wl, args, world, rank, local, dev, steps=args.steps, warmup=args.warmup, layers=args.layers,
+                  depth=depth, want_e2e=not (args.no_e2e or depth),
+                  want_cpu=rank == 0 and world == 1 and not args.no_cpu_baseline, fused=fused)
+    per = None
+    if args.per_workload and not depth and not args.window and world == 1:
+        per = per_workload_runs(args, world, rank, local, dev, wl)
 
     if rank == 0:
-        n_layer_steps = args.steps * L
+        L, B, hq, hkv, d = res["L"], res["B"], res["hq"], res["hkv"], res["d"]
+        steps = args.steps
+        peak, achieved = res["peak"], res["achieved"]
+        kernel = {"auto": "mma" if wl.dtype == "bf16" else "simt"}.get(args.attn_kernel, args.attn_kernel)
+        attn_ms, timed_tot, per_layer = res["attn_ms"], res["timed_tot"], res["per_layer"]
+        launch_timing = ("timed region (CUDA events at its two ends) over its step launches; "
+                         "isolated: an event pair around every launch, in a second pass over the next steps"
+                         if fused else
+                         "attention launches back to back between one event pair (the burst); "
+                         "isolated: an event pair around every launch, in a second pass over the next steps")
         line = {
-            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": t_max_ms / args.steps, "higher_is_better": True,
+            "metric": METRIC, "value": res["value"], "unit": "GB/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": res["t_max_ms"] / steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": {
                 "workload": wl.name, "batch_per_gpu": B, "q_heads": hq, "kv_heads": hkv, "head_dim": d,
-                "window": wl.window, "context": int(ctx.max()) if wl.ctx_range is None else list(wl.ctx_range),
+                "window": wl.window,
+                "context": int(res["ctx"].max()) if wl.ctx_range is None else list(wl.ctx_range),
                 "layers": L, "attn_kernel": kernel, "parallelism": f"replicas x{world}",
-                "l2": f"inputs larger than L2: {L} layer pools, {total_bytes / args.steps / 2**20:.0f} MiB "
+                "l2": f"inputs larger than L2: {L} layer pools, {res['total_bytes'] / steps / 2**20:.0f} MiB "
                       f"retained K/V read per step vs 126 MiB L2",
                 "step": ("per layer: dms_decode_step (append 1 token/seq + attention, one launch)" if fused else
                          "per layer: dms_append (1 token/seq) + dms_decode_attention") +
                         ("; one dms_stats per layer per step" if depth else "; one dms_stats per step"),
             },
-            "decode_steps_per_s_per_layer": n_layer_steps / (t_max_ms * 1e-3),
-            "retained_bytes_per_step": total_bytes / args.steps,
+            "decode_steps_per_s_per_layer": steps * L / (res["t_max_ms"] * 1e-3),
+            "retained_bytes_per_step": res["total_bytes"] / steps,
             "compression_ratio": float(timed_tot[-1, 0] / timed_tot[-1, 1]),
             **({"depth": {"cr_schedule": depth, "layer_cr": [
-                float(x) for x in per_layer[args.warmup + args.steps - 1, :, 0] /
-                per_layer[args.warmup + args.steps - 1, :, 1]]}} if depth else {}),
+                float(x) for x in per_layer[args.warmup + steps - 1, :, 0] /
+                per_layer[args.warmup + steps - 1, :, 1]]}} if depth else {}),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "frac": achieved / peak, "peak_kind": res["peak_kind"],
+                         "frac_nominal": achieved / NOMINAL_HBM_GBS, "peak_nominal": NOMINAL_HBM_GBS,
                          "traffic": profile_traffic(wl.name, kernel,
                                                     "dms_decode_step" if fused else "dms_decode_attention"),
                          "kernel": f"dms_decode_step ({kernel}, append fused)" if fused else
                                    f"dms_decode_attention ({kernel})",
-                         "bytes_per_launch": float(bytes_launch.mean()) if fused else float(bytes_pl.mean()),
-                         "launch_ms": launch_ms, "launch_timing": launch_timing,
+                         "bytes_per_launch": res["bytes_launch"],
+                         "launch_ms": res["launch_ms"], "launch_timing": launch_timing,
                          "launch_ms_isolated": float(attn_ms.mean()),
                          "launch_ms_isolated_p10": float(np.percentile(attn_ms, 10)),
                          "launch_ms_isolated_p90": float(np.percentile(attn_ms, 90)),
-                         "achieved_isolated": achieved_iso, "frac_isolated": achieved_iso / peak,
-                         "launch_ms_burst": burst_ms, "achieved_burst": achieved_burst,
-                         "frac_burst": achieved_burst / peak},
-            "gpu_launches": launches,
-            "clocks": clk.summary(),
+                         "achieved_isolated": res["achieved_iso"], "frac_isolated": res["achieved_iso"] / peak,
+                         "frac_isolated_nominal": res["achieved_iso"] / NOMINAL_HBM_GBS,
+                         "launch_ms_burst": res["burst_ms"], "achieved_burst": res["achieved_burst"],
+                         "frac_burst": res["achieved_burst"] / peak},
+            "gpu_launches": res["launches"],
+            "clocks": res["clocks"],
         }
-        if e2e is not None:
-            line["e2e"] = e2e
-        if cpu is not None:
-            line["cpu_baseline"] = cpu
+        if "e2e" in res:
+            line["e2e"] = res["e2e"]
+        if "cpu" in res:
+            line["cpu_baseline"] = res["cpu"]
+        if per is not None:
+            line["per_workload"] = per
         print(json.dumps(line), flush=True)
 
-    for c in caches:
-        c.close()
     if world > 1:
         dist.destroy_process_group()
 

@@ -14,6 +14,10 @@
  * Reading of the window bound used throughout: position j is visible to
  * the query at step s iff alpha_j == 0 or s - j < w.
  *
+ * The pages define the computation, not an API. Each call below names the
+ * passage it serves; the cache life-cycle and inspection calls, for which
+ * the pages define nothing, say so.
+ *
  * Storage. A *stream* is one (sequence, KV head) pair, stream id =
  * seq_id * num_kv_heads + kv_head. A stream holds its retained tokens in
  * logical slots [0, n); logical slot l lives in physical page
@@ -39,8 +43,13 @@
  *     and *poison* the cache: every later kernel on it does nothing until
  *     dms_cache_reset. Read the word with dms_get_status (syncs).
  *   - One cache must not be used from two streams at the same time. Calls
- *     on one stream run in order; dms_append of a step must precede the
+ *     on one cache run in the order they are made: on one stream, or on
+ *     streams ordered by events. dms_append of a step must precede the
  *     dms_decode_attention that should see that step's token.
+ *   - Different caches may be used from different streams at the same
+ *     time, in any interleaving. No kernel of this library waits on another
+ *     of its CTAs, so a launch finishes with whatever share of the SMs it
+ *     gets, however the device is shared.
  *   - seq_ids inside one call must be distinct.
  */
 #ifndef DMS_H
@@ -86,7 +95,9 @@ typedef struct {
     dms_attn_kernel attn_kernel;   /* decode-attention kernel choice */
 } dms_config;
 
-/* Create a cache on the current CUDA device. Allocates the pool
+/* Create a cache on the current CUDA device (life cycle; the pages define no
+ * API: they fix only that the cache is paged and per head, section 3.2
+ * "Performance Considerations"). Allocates the pool
  * (max_pages * 2 * 16 * head_dim elements), the page tables, the free stack,
  * the per-stream counters and window rings, and the split-K scratch
  * (partials and per-stream counters). Zeroes everything. Syncs.
@@ -94,23 +105,25 @@ typedef struct {
  * an allocation fails (nothing leaks). */
 dms_status dms_cache_create(const dms_config* cfg, dms_cache** out);
 
-/* Free everything. Syncs the device. NULL is accepted. */
+/* Free everything (life cycle; the pages define no API). Syncs the device.
+ * NULL is accepted. */
 dms_status dms_cache_destroy(dms_cache* cache);
 
-/* Return the cache to its freshly created state (all sequences empty, free
- * stack full, status cleared). Pool contents are not cleared. Async. */
+/* Return the cache to its freshly created state: all sequences empty, free
+ * stack full, status cleared (life cycle; the pages define no API). Pool
+ * contents are not cleared. Async. */
 dms_status dms_cache_reset(dms_cache* cache, cudaStream_t stream);
 
 /* Release sequence seq_id (host int): push its pages back on the free stack
  * (KV head ascending, each stream's pages last to first) and clear its
- * counters and window rings. Async. */
+ * counters and window rings (life cycle; the pages define no API). Async. */
 dms_status dms_seq_reset(dms_cache* cache, cudaStream_t stream, int32_t seq_id);
 
 /* Append tokens and apply delayed eviction (paper summary, Method; section
- * 3.2). For every (sequence, KV head) stream of the call and every new token
- * s in position order: retire the token at s - w if it was marked and reuse
- * its slot, else take a fresh slot; write the K and V rows into the pool;
- * record alpha_s.
+ * 3.2: the decision taken at step t acts at step t + w). For every
+ * (sequence, KV head) stream of the call and every new token s in position
+ * order: retire the token at s - w if it was marked and reuse its slot, else
+ * take a fresh slot; write the K and V rows into the pool; record alpha_s.
  *   n_seqs        sequences in this call (host int, >= 0)
  *   seq_ids       device int32 [n_seqs], distinct, each in [0, max_seqs)
  *   cu_tokens     device int32 [n_seqs + 1] prefix offsets of each
@@ -128,10 +141,10 @@ dms_status dms_append(dms_cache* cache, cudaStream_t stream, int32_t n_seqs,
                       const int32_t* seq_ids, const int32_t* cu_tokens, int32_t total_tokens,
                       const void* K, const void* V, const uint8_t* alpha);
 
-/* dms_append with the eviction decisions read from the keys (scope row "alpha
- * from the logit": paper summary, Method: one neuron of the K projection
- * per head is repurposed to give the eviction logit; reading R4 of the
- * design notes: at inference alpha_t = 1 iff that logit is > 0). For every
+/* dms_append with the eviction decisions read from the keys (paper summary,
+ * Method: one neuron of the K projection per head is repurposed to give the
+ * eviction logit). The pages do not say how the logit is binarised at
+ * inference; the library takes alpha = 1 iff the logit is > 0. For every
  * appended token t and KV head h: alpha = 1 iff K[t, h, alpha_channel] > 0
  * (zero and NaN keep the token). K and V are stored as given, the logit
  * channel included. Same bookkeeping and errors as dms_append with those
@@ -140,6 +153,24 @@ dms_status dms_append(dms_cache* cache, cudaStream_t stream, int32_t n_seqs,
 dms_status dms_append_keyed(dms_cache* cache, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                             const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
                             int32_t alpha_channel);
+
+/* Eviction decisions from a designated logit channel of a projection (paper
+ * summary, Method: one neuron of the K or the Q projection per head is
+ * repurposed to give the eviction logit; taken as alpha = 1 iff the logit is
+ * > 0, zero and NaN keep the token). Needs no cache.
+ *   X             device [rows, num_kv_heads * heads_per_kv, head_dim] of
+ *                 dtype: keys (heads_per_kv = 1) or queries (heads_per_kv =
+ *                 g, the GQA group; query heads k*g .. k*g+g-1 belong to KV
+ *                 head k)
+ *   head          host int in [0, heads_per_kv): the designated head of
+ *                 each KV head's group (0 for keys)
+ *   channel       host int in [0, head_dim)
+ *   alpha_out     device uint8 [rows, num_kv_heads]:
+ *                 alpha_out[r, k] = X[r, k * heads_per_kv + head, channel] > 0
+ * The result feeds dms_append's alpha argument. Async. */
+dms_status dms_alpha_from_logit(cudaStream_t stream, const void* X, dms_dtype dtype, int32_t rows,
+                                int32_t num_kv_heads, int32_t heads_per_kv, int32_t head, int32_t head_dim,
+                                int32_t channel, uint8_t* alpha_out);
 
 /* One decode step of GQA attention over the retained tokens (paper summary,
  * Key claims: memory reads dominate decode latency; the mask is never
@@ -159,8 +190,7 @@ dms_status dms_append_keyed(dms_cache* cache, cudaStream_t stream, int32_t n_seq
  * cache's, the call guesses that it has the previous call's streams. It plans
  * from the cache state and starts its first page copies before that kernel has
  * finished (programmatic dependent launch), and checks the guess against
- * seq_ids once it has. Calls on one cache must run in the order they are made:
- * on one stream, or on streams ordered by events. Async. */
+ * seq_ids once it has. Async. */
 dms_status dms_decode_attention(dms_cache* cache, cudaStream_t stream, int32_t n_seqs,
                                 const int32_t* seq_ids, const void* Q, int32_t num_q_heads,
                                 float scale, void* out, dms_dtype out_dtype);
@@ -168,17 +198,19 @@ dms_status dms_decode_attention(dms_cache* cache, cudaStream_t stream, int32_t n
 /* One whole decode step in one launch: dms_append of one token per sequence
  * (cu_tokens = NULL) followed by dms_decode_attention, with the same results:
  * the same bookkeeping bit for bit, and outputs equal up to fp32 rounding
- * order (scope row "fused append + attention", paper summary, Key claims:
- * decode is bound by memory reads, so the step should cost one pass over
- * the retained K/V and one launch).
+ * order (paper summary, Key claims: decode is bound by memory reads and DMS
+ * adds no read or write of the KV cache, so the step should cost one pass
+ * over the retained K/V and one launch).
  * The attention runs over the cache as it was before the step, with the row
  * of the token that leaves at this step masked and the new token taken
  * from K and V; the append's writes go to rows that no part of the launch
- * attends. A cache with more than 1024 streams (max_seqs * num_kv_heads), or
- * whose configuration leaves no shared memory for the step's per-stream
- * state, issues the two launches instead; so does a call on a stream that is
- * being captured into a CUDA graph (the fused launch carries host sequence
- * numbers and cannot be replayed).
+ * attends. The launch reads one copy of the per-stream counts and writes
+ * the other (the cache keeps two and flips between them), so none of its
+ * CTAs waits on another. A cache with more than 1024 streams (max_seqs *
+ * num_kv_heads), or whose configuration leaves no shared memory for the
+ * step's per-stream state, issues the two launches instead; so does a call
+ * on a stream that is being captured into a CUDA graph (the fused launch
+ * carries host sequence numbers and cannot be replayed).
  * Each fused step leaves the next one on the same cache a schedule: every
  * call stream's count, position and leaving slot after it, and the page ids
  * of every CTA's range. The next fused step uses it when no other call has
@@ -188,8 +220,7 @@ dms_status dms_decode_attention(dms_cache* cache, cudaStream_t stream, int32_t n
  * not one of this cache's, it plans and starts its first page copies before
  * that kernel has finished (programmatic dependent launch), on the guess that
  * its seq ids are those of the step that left the schedule; the guess is
- * checked once the previous kernel is done. Calls on one cache must run in
- * the order they are made: on one stream, or on streams ordered by events.
+ * checked once the previous kernel is done.
  * Every kernel of this library that writes a cache lets the next kernel of its
  * stream start only after its own dependency wait; other code that uses
  * programmatic dependent launch on the same stream must do the same (call
@@ -205,10 +236,23 @@ dms_status dms_decode_step(dms_cache* cache, cudaStream_t stream, int32_t n_seqs
                            int32_t num_q_heads, float scale, void* out, dms_dtype out_dtype);
 
 /* dms_decode_step with the eviction decisions read from the keys, as
- * dms_append_keyed: alpha = 1 iff K[b, h, alpha_channel] > 0. */
+ * dms_append_keyed: alpha = 1 iff K[b, h, alpha_channel] > 0 (paper summary,
+ * Method: a repurposed K neuron gives the logit). */
 dms_status dms_decode_step_keyed(dms_cache* cache, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                                  const void* K, const void* V, int32_t alpha_channel, const void* Q,
                                  int32_t num_q_heads, float scale, void* out, dms_dtype out_dtype);
+
+/* dms_decode_step with the eviction decisions read from the step's queries
+ * (paper summary, Method: the repurposed neuron may come from the Q
+ * projection instead). The decision of KV head k is taken from query head
+ * k * g + alpha_head (the designated head of its group):
+ * alpha = 1 iff Q[b, k * g + alpha_head, alpha_channel] > 0.
+ *   alpha_head     host int in [0, g)
+ *   alpha_channel  host int in [0, head_dim) */
+dms_status dms_decode_step_qkeyed(dms_cache* cache, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                                  const void* K, const void* V, const void* Q, int32_t num_q_heads,
+                                  int32_t alpha_head, int32_t alpha_channel, float scale, void* out,
+                                  dms_dtype out_dtype);
 
 /* Retained counts and compression ratios (paper summary, Key claims: CR =
  * tokens seen / tokens kept; each head can land at its own CR). Async;
@@ -221,8 +265,16 @@ dms_status dms_decode_step_keyed(dms_cache* cache, cudaStream_t stream, int32_t 
 dms_status dms_stats(dms_cache* cache, cudaStream_t stream, int32_t* retained, int32_t* seen,
                      float* head_cr, int64_t* totals);
 
-/* Copy the bookkeeping to HOST memory for checking. Syncs the stream. Any
- * pointer may be NULL.
+/* dms_stats with HOST outputs (paper summary, Key claims, as dms_stats).
+ * Syncs the stream. Any pointer may be NULL.
+ *   retained, seen  host int32 [max_seqs * num_kv_heads], as dms_stats
+ *   cr_overall      host double: sum(seen) / sum(retained) over every
+ *                   stream (0 when nothing is retained) */
+dms_status dms_stats_host(dms_cache* cache, cudaStream_t stream, int32_t* retained, int32_t* seen,
+                          double* cr_overall);
+
+/* Copy the bookkeeping to HOST memory for checking (inspection; the pages
+ * define no API). Syncs the stream. Any pointer may be NULL.
  *   page_table  int32 [S * max_pages_per_stream]   (entries >= n_pages are stale)
  *   n_pages, n, pos  int32 [S]
  *   slot_pos    int32 [max_pages * 16]  position stored in each physical slot
@@ -233,8 +285,9 @@ dms_status dms_snapshot(dms_cache* cache, cudaStream_t stream, int32_t* page_tab
                         int32_t* free_list, int32_t* free_count);
 
 /* Gather the retained K and V rows of one stream in logical slot order into
- * device buffers [n, head_dim] of the cache dtype (n from dms_stats or
- * dms_snapshot; rows_cap bounds the copy). Async. */
+ * device buffers [n, head_dim] of the cache dtype (inspection; the pages
+ * define no API). n from dms_stats or dms_snapshot; rows_cap bounds the
+ * copy. Async. */
 dms_status dms_gather_kv(dms_cache* cache, cudaStream_t stream, int32_t seq_id,
                          int32_t kv_head, int32_t rows_cap, void* K_out, void* V_out);
 
@@ -257,7 +310,9 @@ dms_status dms_gather_kv(dms_cache* cache, cudaStream_t stream, int32_t seq_id,
  *
  * The first call on a device (with that device current) looks up the
  * array's device address and sets the kernel's attributes. Make that first
- * call before any stream capture. Later calls reuse the set-up.
+ * call before any stream capture. Later calls reuse the set-up; the launch
+ * plans of the last 8 distinct call shapes (pool, head_dim, dtype, streams,
+ * max_pages) are kept, so alternating shapes prepare nothing again.
  *
  * Every call on a device shares the one array: calls whose kernels may
  * overlap on the GPU (different streams, no ordering between them) race on
@@ -272,14 +327,16 @@ dms_status dms_gather_kv(dms_cache* cache, cudaStream_t stream, int32_t seq_id,
  *     kv_pool      device [max_pages][2][16][head_dim] of dtype, 16-B aligned:
  *                  per page 16 K rows then 16 V rows
  *     page_table   device int32 [max_seqs * num_kv_heads][max_pages_per_stream]
- *     retained     device int32 [max_seqs * num_kv_heads]: n of each stream,
- *                  in [0, 16 * max_pages_per_stream]; its tokens sit in
- *                  logical slots [0, n). Larger or negative counts are not
- *                  checked and make the kernel read past the page table.
+ *     retained     device int32 [max_seqs * num_kv_heads]: n of each stream;
+ *                  its tokens sit in logical slots [0, n). A count outside
+ *                  [0, 16 * max_pages_per_stream] is clamped into it: a larger
+ *                  one attends every slot the page table addresses, a negative
+ *                  one attends nothing (zeros out).
  *   seq_ids, Q, num_q_heads, scale, out, out_dtype: as dms_decode_attention.
  * Device-side checks (a seq id outside [0, max_seqs), a page id outside
- * [0, max_pages)) skip the bad access, but no later call reports them: the
- * outputs of those streams are then unspecified. Async. */
+ * [0, max_pages), a clamped count) skip or bound the bad access, but no
+ * later call reports them: the outputs of those streams are then
+ * unspecified, except as the clamp above states. Async. */
 #define DMS_NOALLOC_MAX_STREAMS 512
 #define DMS_NOALLOC_MAX_PIECES 1024
 
@@ -299,7 +356,8 @@ dms_status dms_decode_attention_noalloc(cudaStream_t stream, const dms_paged_kv*
                                         const int32_t* seq_ids, const void* Q, int32_t num_q_heads,
                                         float scale, void* out, dms_dtype out_dtype);
 
-/* Sync the stream and return the latched device status (DMS_OK if none). */
+/* Sync the stream and return the latched device status, DMS_OK if none
+ * (failure detection; the pages define no API). */
 dms_status dms_get_status(dms_cache* cache, cudaStream_t stream);
 
 /* Static description of a status code. */
@@ -320,7 +378,7 @@ const char* dms_status_string(dms_status s);
 dms_status dms_selftest_bounded_waits(dms_cache* cache, cudaStream_t stream, int32_t* timed_out);
 
 /* Kernel launches issued by the library since the cache was created (host
- * counter, for accounting). */
+ * counter, for accounting; the pages define no API). */
 int64_t dms_launch_count(const dms_cache* cache);
 
 #ifdef __cplusplus

@@ -21,7 +21,7 @@ import torch
 from . import _native
 from ._native import DmsError
 
-__all__ = ["DmsCache", "DmsError", "decode_attention_noalloc"]
+__all__ = ["DmsCache", "DmsError", "decode_attention_noalloc", "alpha_from_logit"]
 
 _DTYPES = {torch.bfloat16: _native.DMS_BF16, torch.float32: _native.DMS_F32}
 _KERNELS = {"auto": _native.DMS_ATTN_AUTO, "simt": _native.DMS_ATTN_SIMT, "mma": _native.DMS_ATTN_MMA}
@@ -115,15 +115,23 @@ class DmsCache:
 
     def decode_step(self, seq_ids: torch.Tensor, K: torch.Tensor, V: torch.Tensor, alpha: torch.Tensor | None,
                     Q: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None,
-                    out_dtype: torch.dtype | None = None, alpha_channel: int | None = None) -> torch.Tensor:
+                    out_dtype: torch.dtype | None = None, alpha_channel: int | None = None,
+                    alpha_head: int | None = None) -> torch.Tensor:
         """One decode step in one launch: append one token per sequence (K, V [B, Hkv, d],
-        alpha uint8 [B, Hkv], or alpha_channel: alpha = K[..., alpha_channel] > 0) and
+        alpha uint8 [B, Hkv], or alpha_channel: alpha = K[..., alpha_channel] > 0, or with
+        alpha_head as well: alpha = Q[:, kv * g + alpha_head, alpha_channel] > 0) and
         attend with Q [B, Hq, d] -> out [B, Hq, d]."""
         b, hq, d = Q.shape
         if scale is None:
             scale = 1.0 / math.sqrt(d)
         if out is None:
             out = torch.empty((b, hq, d), dtype=out_dtype or Q.dtype, device=Q.device)
+        if alpha_channel is not None and alpha_head is not None:
+            _native.check(self.lib.dms_decode_step_qkeyed(self._h, _stream(), int(seq_ids.numel()), _ptr(seq_ids),
+                                                          _ptr(K), _ptr(V), _ptr(Q), hq, int(alpha_head),
+                                                          int(alpha_channel), float(scale), _ptr(out),
+                                                          _DTYPES[out.dtype]), "dms_decode_step_qkeyed")
+            return out
         if alpha_channel is not None:
             _native.check(self.lib.dms_decode_step_keyed(self._h, _stream(), int(seq_ids.numel()), _ptr(seq_ids),
                                                          _ptr(K), _ptr(V), int(alpha_channel), _ptr(Q), hq,
@@ -145,6 +153,17 @@ class DmsCache:
         tot = torch.empty(2, dtype=torch.int64, device=dev)
         _native.check(self.lib.dms_stats(self._h, _stream(), _ptr(r), _ptr(s), _ptr(cr), _ptr(tot)), "dms_stats")
         return {"retained": r, "seen": s, "head_cr": cr, "totals": tot}
+
+    def stats_host(self) -> dict:
+        """Host copies of the per-stream counts and the overall compression ratio
+        (wraps dms_stats_host; syncs the stream)."""
+        import numpy as np
+        r = np.empty(self.streams, dtype=np.int32)
+        s = np.empty(self.streams, dtype=np.int32)
+        cr = ctypes.c_double()
+        _native.check(self.lib.dms_stats_host(self._h, _stream(), r.ctypes.data, s.ctypes.data, ctypes.byref(cr)),
+                      "dms_stats_host")
+        return {"retained": r, "seen": s, "cr_overall": cr.value}
 
     def snapshot(self) -> dict:
         """Host copies of the bookkeeping (syncs the stream)."""
@@ -213,4 +232,22 @@ def decode_attention_noalloc(kv_pool: torch.Tensor, page_table: torch.Tensor, re
     _native.check(lib.dms_decode_attention_noalloc(_stream(), ctypes.byref(kv), int(seq_ids.numel()),
                                                    _ptr(seq_ids), _ptr(Q), hq, float(scale), _ptr(out),
                                                    _DTYPES[out.dtype]), "dms_decode_attention_noalloc")
+    return out
+
+
+def alpha_from_logit(X: torch.Tensor, num_kv_heads: int, channel: int, head: int = 0,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """Eviction decisions from the sign of a designated projection channel (wraps
+    ``dms_alpha_from_logit``). X [rows, num_kv_heads * h, d] holds keys (h = 1) or
+    queries (h = g, and ``head`` picks one query head of each KV head's group);
+    returns uint8 [rows, num_kv_heads]: 1 iff X[r, k * h + head, channel] > 0."""
+    lib = _native.load()
+    rows, heads, d = X.shape
+    if heads % num_kv_heads:
+        raise ValueError("the head count of X must be a multiple of num_kv_heads")
+    if out is None:
+        out = torch.empty((rows, num_kv_heads), dtype=torch.uint8, device=X.device)
+    _native.check(lib.dms_alpha_from_logit(_stream(), _ptr(X), _DTYPES[X.dtype], rows, num_kv_heads,
+                                           heads // num_kv_heads, int(head), d, int(channel), _ptr(out)),
+                  "dms_alpha_from_logit")
     return out

@@ -9,7 +9,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdms.so")
+# DMS_LIBRARY=debug selects the build with device-side bounds checks
+# (libdms_debug.so); the default is libdms.so.
+LIB_PATH = os.path.join(_HERE, "libdms_debug.so" if os.environ.get("DMS_LIBRARY") == "debug" else "libdms.so")
 
 DMS_OK = 0
 DMS_ERR_INVALID = 1
@@ -30,7 +32,8 @@ DMS_ATTN_MMA = 2
 EXPORTS = ("dms_cache_create", "dms_cache_destroy", "dms_cache_reset", "dms_seq_reset", "dms_append",
            "dms_decode_attention", "dms_stats", "dms_snapshot", "dms_gather_kv", "dms_get_status",
            "dms_status_string", "dms_launch_count", "dms_decode_attention_noalloc", "dms_decode_step",
-           "dms_append_keyed", "dms_decode_step_keyed", "dms_selftest_bounded_waits")
+           "dms_append_keyed", "dms_decode_step_keyed", "dms_selftest_bounded_waits",
+           "dms_decode_step_qkeyed", "dms_alpha_from_logit", "dms_stats_host")
 
 DMS_NOALLOC_MAX_STREAMS = 512
 DMS_NOALLOC_MAX_PIECES = 1024
@@ -100,6 +103,8 @@ def load() -> ctypes.CDLL:
     L.dms_decode_attention.restype = st
     L.dms_stats.argtypes = [p, p, p, p, p, p]
     L.dms_stats.restype = st
+    L.dms_stats_host.argtypes = [p, p, p, p, ctypes.POINTER(ctypes.c_double)]
+    L.dms_stats_host.restype = st
     L.dms_snapshot.argtypes = [p, p, p, p, p, p, p, p, p]
     L.dms_snapshot.restype = st
     L.dms_gather_kv.argtypes = [p, p, i32, i32, i32, p, p]
@@ -118,6 +123,10 @@ def load() -> ctypes.CDLL:
     L.dms_append_keyed.restype = st
     L.dms_decode_step_keyed.argtypes = [p, p, i32, p, p, p, i32, p, i32, ctypes.c_float, p, ctypes.c_int]
     L.dms_decode_step_keyed.restype = st
+    L.dms_decode_step_qkeyed.argtypes = [p, p, i32, p, p, p, p, i32, i32, i32, ctypes.c_float, p, ctypes.c_int]
+    L.dms_decode_step_qkeyed.restype = st
+    L.dms_alpha_from_logit.argtypes = [p, p, ctypes.c_int, i32, i32, i32, i32, i32, i32, p]
+    L.dms_alpha_from_logit.restype = st
     L.dms_decode_attention_noalloc.argtypes = [p, ctypes.POINTER(DmsPagedKv), i32, p, p, i32, ctypes.c_float, p,
                                                ctypes.c_int]
     L.dms_decode_attention_noalloc.restype = st

@@ -22,7 +22,10 @@ struct dms_cache {
   dms::AttnPlan plan{};
   dms::AttnPlan step_plan{};   // fused decode step (append + attention in one launch)
   bool has_step = false;       // else dms_decode_step issues the two launches
-  uint64_t step_launches = 0;  // fused steps launched since the counters were last cleared
+  // State parity after every launch issued so far (see dms::kCtrlPar): it flips
+  // with every fused step, the only kernel that changes it. Eager launches take
+  // it from here; a launch into a stream under capture reads the device word.
+  int par = 0;
   // Schedules fused steps leave for the next one (see dms::NextPlan): the tag of
   // the last fused launch, and the tag the next fused launch may trust (0 once
   // any other call has changed the cache).
@@ -33,6 +36,7 @@ struct dms_cache {
   // and the number of attention launches so far (its parity picks the buffers).
   int32_t* attn_guess = nullptr;
   uint64_t attn_launches = 0;
+  int64_t* totals_dev = nullptr;   // {sum(seen), sum(retained)} for dms_stats_host
   int64_t launches = 0;
   bool poisoned = false;   // a device error was observed by dms_get_status
 };
@@ -97,6 +101,29 @@ bool note_launch(const dms_cache* c, int device, cudaStream_t s) {
 
 dms_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DMS_OK : DMS_ERR_CUDA; }
 
+// Whether `s` is being captured into a CUDA graph (-1: the query failed).
+int capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &capture) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return capture != cudaStreamCaptureStatusNone ? 1 : 0;
+}
+
+// Retained counts for an attention launch of this cache on `s`.
+dms::AttnCounts counts_for(const dms_cache* h, cudaStream_t s) {
+  return dms::AttnCounts{h->dv.n, h->dv.S, capturing(s) == 0 ? h->par : -1};
+}
+
+// Where an append or a fused step takes its eviction decisions from.
+dms::AlphaSrc alpha_src(const dms_cache* h, const void* K, const void* Q, int hq, const dms::AlphaChoice& c) {
+  const dms::Dev& dv = h->dv;
+  if (c.channel < 0) return dms::alpha_given(c.alpha, dv.hkv);
+  if (c.q_head < 0) return dms::alpha_from_keys(K, dv.hkv, dv.d, c.channel, dv.elem_bytes);
+  return dms::alpha_from_queries(Q, dv.hkv, hq / dv.hkv, dv.d, c.q_head, c.channel, dv.elem_bytes);
+}
+
 // Every call must run with the cache's device current.
 dms_status check_device(const dms_cache* c) {
   int dev = -1;
@@ -130,15 +157,16 @@ void free_next(dms::NextPlan& np) {
   np = dms::NextPlan{};
 }
 
-// Buffers of the schedules a fused step leaves for the next one: one entry per
-// stream, and per tag parity one page list per CTA of the step's grid, long
-// enough for any range (a call holds at most max_pages pages).
+// Buffers of the schedules a fused step leaves for the next one: per tag
+// parity, one entry per stream and one page list per CTA of the step's grid,
+// long enough for any range (a call holds at most max_pages pages).
 cudaError_t alloc_next(const dms::Dev& dv, int grid, dms::NextPlan* np) {
   np->cap = (int)std::max<int64_t>(1, ((int64_t)dv.max_pages + grid - 1) / grid);
-  cudaError_t e = alloc(&np->entry, (size_t)dv.S);
+  np->S = dv.S;
+  cudaError_t e = alloc(&np->entry, (size_t)2 * dv.S);
   if (e == cudaSuccess) e = alloc(&np->hdr, (size_t)2 * grid * 2);
   if (e == cudaSuccess) e = alloc(&np->list, (size_t)2 * grid * np->cap);
-  if (e == cudaSuccess) e = cudaMemset(np->entry, 0, (size_t)dv.S * sizeof(dms::PlanEntry));
+  if (e == cudaSuccess) e = cudaMemset(np->entry, 0, (size_t)2 * dv.S * sizeof(dms::PlanEntry));
   if (e == cudaSuccess) e = cudaMemset(np->hdr, 0, (size_t)2 * grid * 2 * sizeof(int4));
   return e;
 }
@@ -161,7 +189,7 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
   if (c.attn_kernel != DMS_ATTN_AUTO && c.attn_kernel != DMS_ATTN_SIMT && c.attn_kernel != DMS_ATTN_MMA)
     return DMS_ERR_INVALID;
   if (c.attn_kernel == DMS_ATTN_MMA && c.dtype != DMS_BF16) return DMS_ERR_INVALID;
-  if ((int64_t)c.max_seqs * c.num_kv_heads * c.window > (int64_t)1 << 31) return DMS_ERR_INVALID;
+  if ((int64_t)c.max_seqs * c.num_kv_heads * ((int64_t)c.window + 1) > (int64_t)1 << 31) return DMS_ERR_INVALID;
   if ((int64_t)c.max_seqs * c.num_kv_heads * c.max_pages_per_stream > (int64_t)1 << 31) return DMS_ERR_INVALID;
 
   dms_cache* h = new (std::nothrow) dms_cache();
@@ -185,11 +213,11 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
   const size_t S = dv.S;
   cudaError_t e = cudaSuccess;
   auto step = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
-  step(alloc(&dv.pos, S));
-  step(alloc(&dv.n, S));
+  step(alloc(&dv.pos, 2 * S));   // one copy per state parity
+  step(alloc(&dv.n, 2 * S));
   step(alloc(&dv.n_pages, S));
   step(alloc(&dv.page_table, S * dv.mps));
-  step(alloc(&dv.ring, S * dv.w));
+  step(alloc(&dv.ring, S * ((size_t)dv.w + 1)));
   step(alloc(&dv.slot_pos, (size_t)dv.max_pages * dms::kPage));
   step(alloc(&dv.free_list, (size_t)dv.max_pages));
   step(alloc(&dv.ctrl, (size_t)dms::kCtrlWords));
@@ -206,8 +234,10 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
   }
   if (e == cudaSuccess && h->has_step) e = alloc_next(dv, h->step_plan.grid, &h->next);
   if (e == cudaSuccess) e = alloc(&h->attn_guess, (size_t)2 * (1 + c.max_seqs));
+  if (e == cudaSuccess) e = alloc(&h->totals_dev, (size_t)2);
   if (e == cudaSuccess) e = cudaMemset(h->attn_guess, 0xff, (size_t)2 * (1 + c.max_seqs) * sizeof(int32_t));
   const int grid = h->has_step && h->step_plan.grid > h->plan.grid ? h->step_plan.grid : h->plan.grid;
+  dv.part_slots = grid + dv.S;
   if (e == cudaSuccess) e = alloc(&dv.part, ((size_t)grid + dv.S) * dms::kMaxGroup * (dv.d + 2));
   if (e == cudaSuccess) e = cudaMemset(dv.kv, 0, (size_t)dv.max_pages * 2 * dms::kPage * dv.d * dv.elem_bytes);
   if (e == cudaSuccess) e = cudaMemset(dv.page_table, 0xff, S * dv.mps * sizeof(int32_t));
@@ -218,6 +248,7 @@ dms_status dms_cache_create(const dms_config* cfg, dms_cache** out) {
     free_all(dv);
     free_next(h->next);
     if (h->attn_guess) cudaFree(h->attn_guess);
+    if (h->totals_dev) cudaFree(h->totals_dev);
     delete h;
     cudaGetLastError();
     return e == cudaErrorInvalidValue ? DMS_ERR_INVALID : DMS_ERR_CUDA;
@@ -237,6 +268,7 @@ dms_status dms_cache_destroy(dms_cache* h) {
   free_all(h->dv);
   free_next(h->next);
   if (h->attn_guess) cudaFree(h->attn_guess);
+  if (h->totals_dev) cudaFree(h->totals_dev);
   if (prev >= 0) cudaSetDevice(prev);
   delete h;
   return from_cuda(e);
@@ -249,11 +281,11 @@ dms_status dms_cache_reset(dms_cache* h, cudaStream_t stream) {
   h->trust_tag = 0;
   note_launch(h, h->device, stream);
   cudaError_t e = cudaMemsetAsync(h->dv.page_table, 0xff, (size_t)h->dv.S * h->dv.mps * sizeof(int32_t), stream);
-  if (e == cudaSuccess) e = dms::launch_init_state(h->dv, stream);   // clears the step counter too
+  if (e == cudaSuccess) e = dms::launch_init_state(h->dv, stream);   // state parity 0 again
   h->launches += 1;
   if (e == cudaSuccess) {
     h->poisoned = false;
-    h->step_launches = 0;
+    h->par = 0;
   }
   return from_cuda(e);
 }
@@ -279,7 +311,7 @@ cudaError_t attention_impl(dms_cache* h, cudaStream_t stream, bool early, int32_
   const dms::AttnGuess guess{h->attn_guess + ((k + 1) & 1) * stride, h->attn_guess + (k & 1) * stride,
                              early && k > 0};
   const cudaError_t e = dms::launch_attention(h->dv, h->plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
-                                              out_dtype == DMS_F32, guess);
+                                              out_dtype == DMS_F32, counts_for(h, stream), guess);
   if (e == cudaSuccess) h->attn_launches += 1;
   return e;
 }
@@ -287,6 +319,7 @@ cudaError_t attention_impl(dms_cache* h, cudaStream_t stream, bool early, int32_
 dms_status append_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
                        const int32_t* cu_tokens, int32_t total_tokens, const void* K, const void* V,
                        const uint8_t* alpha, int32_t alpha_channel) {
+  const dms::AlphaChoice choice{alpha, alpha_channel, -1};
   if (!h || n_seqs < 0 || n_seqs > h->cfg.max_seqs || total_tokens < 0) return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
   if (alpha_channel >= h->cfg.head_dim) return DMS_ERR_INVALID;
@@ -299,41 +332,41 @@ dms_status append_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const 
   note_launch(h, h->device, stream);
   if (cu_tokens == nullptr) {
     if (total_tokens != n_seqs) return DMS_ERR_INVALID;
-    e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, &launches);
+    e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha_src(h, K, nullptr, 0, choice),
+                                  &launches);
   } else {
-    e = dms::launch_append_bulk(h->dv, stream, n_seqs, seq_ids, cu_tokens, total_tokens, K, V, alpha,
-                                alpha_channel, &launches);
+    e = dms::launch_append_bulk(h->dv, stream, n_seqs, seq_ids, cu_tokens, total_tokens, K, V,
+                                alpha_src(h, K, nullptr, 0, choice), &launches);
   }
   h->launches += launches;
   return from_cuda(e);
 }
 
 dms_status step_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids, const void* K,
-                     const void* V, const uint8_t* alpha, int32_t alpha_channel, const void* Q, int32_t num_q_heads,
+                     const void* V, const dms::AlphaChoice& choice, const void* Q, int32_t num_q_heads,
                      float scale, void* out, dms_dtype out_dtype) {
   if (!h || n_seqs < 0 || n_seqs > h->cfg.max_seqs) return DMS_ERR_INVALID;
   if (dms_status s = check_usable(h)) return s;
   if (num_q_heads < h->cfg.num_kv_heads || num_q_heads % h->cfg.num_kv_heads != 0) return DMS_ERR_INVALID;
   if (num_q_heads / h->cfg.num_kv_heads > dms::kMaxGroup) return DMS_ERR_INVALID;
   if (out_dtype != DMS_BF16 && out_dtype != DMS_F32) return DMS_ERR_INVALID;
-  if (alpha_channel >= h->cfg.head_dim) return DMS_ERR_INVALID;
+  if (choice.channel >= h->cfg.head_dim) return DMS_ERR_INVALID;
+  if (choice.channel >= 0 && choice.q_head >= num_q_heads / h->cfg.num_kv_heads) return DMS_ERR_INVALID;
   if (n_seqs == 0) return DMS_OK;
-  if (!seq_ids || !K || !V || (alpha_channel < 0 && !alpha) || !Q || !out) return DMS_ERR_INVALID;
+  if (!seq_ids || !K || !V || (choice.channel < 0 && !choice.alpha) || !Q || !out) return DMS_ERR_INVALID;
   if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(out)) return DMS_ERR_INVALID;
-  // A fused launch carries host sequence numbers (the launch index its
-  // grid-wide counter is checked against, the schedule tags), so a graph
-  // replay of it would be wrong: under stream capture the step is issued as
-  // the two launches, which replay as they were captured.
-  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess) {
-    cudaGetLastError();
-    return DMS_ERR_CUDA;
-  }
-  if (!h->has_step || capture != cudaStreamCaptureStatusNone) {
+  // A fused launch carries host sequence numbers (the state parity it flips,
+  // the schedule tags), so a graph replay of it would be wrong: under stream
+  // capture the step is issued as the two launches, which read the parity from
+  // the device and replay as they were captured.
+  const int capture = capturing(stream);
+  if (capture < 0) return DMS_ERR_CUDA;
+  if (!h->has_step || capture != 0) {
     h->trust_tag = 0;
     note_launch(h, h->device, stream);
     int launches = 0;
-    cudaError_t e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, &launches);
+    cudaError_t e = dms::launch_append_decode(h->dv, stream, n_seqs, seq_ids, K, V,
+                                              alpha_src(h, K, Q, num_q_heads, choice), &launches);
     h->launches += launches;
     if (e != cudaSuccess) return DMS_ERR_CUDA;
     h->launches += 1;
@@ -343,11 +376,11 @@ dms_status step_impl(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const in
   h->launches += 1;
   const uint64_t tag = ++h->step_tags;   // consecutive with trust_tag whenever that is set
   const bool early = note_launch(h, h->device, stream);
-  const cudaError_t e = dms::launch_step(h->dv, h->step_plan, stream, n_seqs, seq_ids, K, V, alpha, alpha_channel, Q,
-                                         num_q_heads, scale, out, out_dtype == DMS_F32, h->step_launches, h->next,
+  const cudaError_t e = dms::launch_step(h->dv, h->step_plan, stream, n_seqs, seq_ids, K, V, choice, Q,
+                                         num_q_heads, scale, out, out_dtype == DMS_F32, h->par, h->next,
                                          h->trust_tag, tag, early);
   h->trust_tag = e == cudaSuccess ? tag : 0;
-  if (e == cudaSuccess) h->step_launches += 1;
+  if (e == cudaSuccess) h->par ^= 1;   // the step writes the other copy of the state and flips the parity
   return from_cuda(e);
 }
 
@@ -388,7 +421,8 @@ dms_status dms_decode_step(dms_cache* h, cudaStream_t stream, int32_t n_seqs, co
                            const void* K, const void* V, const uint8_t* alpha, const void* Q, int32_t num_q_heads,
                            float scale, void* out, dms_dtype out_dtype) {
   const CallRange range("dms_decode_step");
-  return step_impl(h, stream, n_seqs, seq_ids, K, V, alpha, -1, Q, num_q_heads, scale, out, out_dtype);
+  return step_impl(h, stream, n_seqs, seq_ids, K, V, dms::AlphaChoice{alpha, -1, -1}, Q, num_q_heads, scale, out,
+                   out_dtype);
 }
 
 dms_status dms_decode_step_keyed(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
@@ -396,7 +430,33 @@ dms_status dms_decode_step_keyed(dms_cache* h, cudaStream_t stream, int32_t n_se
                                  int32_t num_q_heads, float scale, void* out, dms_dtype out_dtype) {
   const CallRange range("dms_decode_step_keyed");
   if (alpha_channel < 0) return DMS_ERR_INVALID;
-  return step_impl(h, stream, n_seqs, seq_ids, K, V, nullptr, alpha_channel, Q, num_q_heads, scale, out, out_dtype);
+  return step_impl(h, stream, n_seqs, seq_ids, K, V, dms::AlphaChoice{nullptr, alpha_channel, -1}, Q, num_q_heads,
+                   scale, out, out_dtype);
+}
+
+dms_status dms_decode_step_qkeyed(dms_cache* h, cudaStream_t stream, int32_t n_seqs, const int32_t* seq_ids,
+                                  const void* K, const void* V, const void* Q, int32_t num_q_heads,
+                                  int32_t alpha_head, int32_t alpha_channel, float scale, void* out,
+                                  dms_dtype out_dtype) {
+  const CallRange range("dms_decode_step_qkeyed");
+  if (alpha_channel < 0 || alpha_head < 0) return DMS_ERR_INVALID;
+  return step_impl(h, stream, n_seqs, seq_ids, K, V, dms::AlphaChoice{nullptr, alpha_channel, alpha_head}, Q,
+                   num_q_heads, scale, out, out_dtype);
+}
+
+dms_status dms_alpha_from_logit(cudaStream_t stream, const void* X, dms_dtype dtype, int32_t rows,
+                                int32_t num_kv_heads, int32_t heads_per_kv, int32_t head, int32_t head_dim,
+                                int32_t channel, uint8_t* alpha_out) {
+  const CallRange range("dms_alpha_from_logit");
+  if (dtype != DMS_BF16 && dtype != DMS_F32) return DMS_ERR_INVALID;
+  if (rows < 0 || num_kv_heads < 1 || heads_per_kv < 1 || head < 0 || head >= heads_per_kv) return DMS_ERR_INVALID;
+  if (head_dim < 1 || channel < 0 || channel >= head_dim) return DMS_ERR_INVALID;
+  if ((int64_t)num_kv_heads * heads_per_kv * head_dim > (int64_t)1 << 30) return DMS_ERR_INVALID;
+  if (rows == 0) return DMS_OK;
+  if (!X || !alpha_out) return DMS_ERR_INVALID;
+  const int eb = dtype == DMS_BF16 ? 2 : 4;
+  const dms::AlphaSrc src = dms::alpha_from_queries(X, num_kv_heads, heads_per_kv, head_dim, head, channel, eb);
+  return from_cuda(dms::launch_alpha_from_logit(stream, src, rows, alpha_out));
 }
 
 dms_status dms_stats(dms_cache* h, cudaStream_t stream, int32_t* retained, int32_t* seen, float* head_cr,
@@ -410,6 +470,28 @@ dms_status dms_stats(dms_cache* h, cudaStream_t stream, int32_t* retained, int32
   return from_cuda(dms::launch_stats(h->dv, stream, retained, seen, head_cr, totals));
 }
 
+dms_status dms_stats_host(dms_cache* h, cudaStream_t stream, int32_t* retained, int32_t* seen, double* cr_overall) {
+  const CallRange range("dms_stats_host");
+  if (!h) return DMS_ERR_INVALID;
+  if (dms_status s = check_usable(h)) return s;
+  const dms::Dev& dv = h->dv;
+  const size_t S = dv.S;
+  int64_t tot[2] = {0, 0};
+  h->launches += 1;
+  cudaError_t e = dms::launch_stats(dv, stream, nullptr, nullptr, nullptr, h->totals_dev);
+  // The counts of the current state parity: the host's, since the stream's work
+  // is ordered and this call syncs it.
+  if (e == cudaSuccess && retained)
+    e = cudaMemcpyAsync(retained, dv.n + (size_t)h->par * S, S * sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess && seen)
+    e = cudaMemcpyAsync(seen, dv.pos + (size_t)h->par * S, S * sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(tot, h->totals_dev, sizeof(tot), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return DMS_ERR_CUDA;
+  if (cr_overall) *cr_overall = tot[1] > 0 ? (double)tot[0] / (double)tot[1] : 0.0;
+  return DMS_OK;
+}
+
 dms_status dms_snapshot(dms_cache* h, cudaStream_t stream, int32_t* page_table, int32_t* n_pages, int32_t* n,
                         int32_t* pos, int32_t* slot_pos, int32_t* free_list, int32_t* free_count) {
   const CallRange range("dms_snapshot");
@@ -421,13 +503,15 @@ dms_status dms_snapshot(dms_cache* h, cudaStream_t stream, int32_t* page_table, 
   auto cp = [&](void* dst, const void* src, size_t bytes) {
     if (dst && e == cudaSuccess) e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, stream);
   };
+  // The current copies of the counts: the stream's work is eager and ordered,
+  // so the host's parity is the device's once the copies run.
   cp(page_table, dv.page_table, S * dv.mps * sizeof(int32_t));
   cp(n_pages, dv.n_pages, S * sizeof(int32_t));
-  cp(n, dv.n, S * sizeof(int32_t));
-  cp(pos, dv.pos, S * sizeof(int32_t));
+  cp(n, dv.n + (size_t)h->par * S, S * sizeof(int32_t));
+  cp(pos, dv.pos + (size_t)h->par * S, S * sizeof(int32_t));
   cp(slot_pos, dv.slot_pos, (size_t)dv.max_pages * dms::kPage * sizeof(int32_t));
   cp(free_list, dv.free_list, (size_t)dv.max_pages * sizeof(int32_t));
-  cp(free_count, dv.ctrl + dms::kCtrlFree, sizeof(int32_t));
+  cp(free_count, dv.ctrl + dms::kCtrlFree + h->par, sizeof(int32_t));
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   return from_cuda(e);
 }
@@ -449,11 +533,14 @@ dms_status dms_get_status(dms_cache* h, cudaStream_t stream) {
   const CallRange range("dms_get_status");
   if (!h) return DMS_ERR_INVALID;
   if (dms_status s = check_device(h)) return s;
-  int32_t word = 0;
-  cudaError_t e = cudaMemcpyAsync(&word, h->dv.ctrl + dms::kCtrlStatus, sizeof(word), cudaMemcpyDeviceToHost,
-                                  stream);
+  // The common status word, then the errors the fused steps latched (by parity).
+  int32_t words[dms::kCtrlWords] = {};
+  cudaError_t e = cudaMemcpyAsync(words, h->dv.ctrl, sizeof(words), cudaMemcpyDeviceToHost, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return DMS_ERR_CUDA;
+  int32_t word = words[dms::kCtrlStatus];
+  if (word == DMS_OK) word = words[dms::kCtrlStepErr];
+  if (word == DMS_OK) word = words[dms::kCtrlStepErr + 1];
   if (word != DMS_OK) h->poisoned = true;
   return (dms_status)word;
 }

@@ -8,6 +8,8 @@
 // is exactly s - w, so appending s either reuses the slot of s - w (marked)
 // or takes a fresh slot. Slots [0, n) therefore stay dense and no validity
 // bitmap or mask is ever stored.
+#include <algorithm>
+
 #include "dms_internal.cuh"
 
 namespace dms {
@@ -64,8 +66,10 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
   grid_dependency_wait();
   grid_dependents_launch();
 
-  // ---- round trip 1
-  const int fc = *reinterpret_cast<const volatile int32_t*>(&dv.ctrl[kCtrlFree]);
+  // ---- round trip 1 (the free-stack depth of both parities, picked once the
+  // parity word is in)
+  const int par = read_par(dv.ctrl);
+  const int fc0 = read_word(&dv.ctrl[kCtrlFree]), fc1 = read_word(&dv.ctrl[kCtrlFree + 1]);
   auto item_src = [&](int t) -> const uint4* {
     const int i = t / (2 * chunks), which = (t / chunks) & 1, c = t % chunks;
     return reinterpret_cast<const uint4*>((which ? V : K) + (size_t)i * row_bytes) + c;
@@ -88,6 +92,8 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
   int seq, al;
   load_ids(tid, seq, al);
   if (__syncthreads_or(tid == 0 && read_status(dv.ctrl) != 0)) return;   // poisoned cache
+  const Cur cs = cur_state(dv, par);
+  const int fc = par ? fc1 : fc0;
 
   // A call with more streams than threads learns its total page demand
   // first, so that an exhausted pool fails every stream that needs a page.
@@ -100,8 +106,8 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
       bool need = false;
       if (sq >= 0 && sq < dv.max_seqs) {
         const int st = sq * dv.hkv + (r0 + tid) % dv.hkv;
-        const int s = dv.pos[st], nn = dv.n[st];
-        const int r = dv.ring[(size_t)st * dv.w + (s % dv.w)];
+        const int s = cs.pos[st], nn = cs.n[st];
+        const int r = dv.ring[ring_leaving(dv, st, s)];
         need = !((s >= dv.w) && (r & 1)) && (nn % kPage) == 0 && nn / kPage < dv.mps;
       }
       demand += __syncthreads_count(need);
@@ -118,11 +124,10 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     const bool good = live && seq >= 0 && seq < dv.max_seqs;
     if (live && !good) latch(dv.ctrl, DMS_ERR_BAD_SEQ);
     const int st = good ? seq * dv.hkv + i % dv.hkv : 0;
-    const int s = good ? dv.pos[st] : 0;
-    const int nn = good ? dv.n[st] : 0;
+    const int s = good ? cs.pos[st] : 0;
+    const int nn = good ? cs.n[st] : 0;
     // ---- round trip 3
-    int32_t* rp = dv.ring + (size_t)st * dv.w + (s % dv.w);
-    const int r = good ? *rp : 0;
+    const int r = good ? dv.ring[ring_leaving(dv, st, s)] : 0;
     const bool retire = good && (s >= dv.w) && (r & 1);   // token s - w leaves now
     const int slot = retire ? (r >> 1) : nn;
     const int lp = slot / kPage;
@@ -145,9 +150,10 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     int page = -1;
     if (go) {
       if (need) {
-        page = dv.free_list[fc - 1 - (popped + rank)];
+        if (in_bounds(fc - 1 - (popped + rank), dv.max_pages, dv.ctrl)) page = dv.free_list[fc - 1 - (popped + rank)];
+        else go = false;
       } else {
-        page = dv.page_table[(size_t)st * dv.mps + lp];
+        page = in_bounds(lp, dv.mps, dv.ctrl) ? dv.page_table[(size_t)st * dv.mps + lp] : -1;
         if (page < 0 || page >= dv.max_pages) {
           latch(dv.ctrl, DMS_ERR_INVALID);
           go = false;
@@ -160,16 +166,17 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
         dv.page_table[(size_t)st * dv.mps + lp] = page;
         dv.n_pages[st] = lp + 1;
       }
-      if (!retire) dv.n[st] = slot + 1;
+      if (!retire) cs.n[st] = slot + 1;
       phys = page * kPage + slot % kPage;
-      *rp = (slot << 1) | al;
-      dv.pos[st] = s + 1;
-      dv.slot_pos[phys] = s;
+      dv.ring[ring_at(dv, st, s)] = (slot << 1) | al;
+      cs.pos[st] = s + 1;
+      if (in_bounds(phys, (long long)dv.max_pages * kPage, dv.ctrl)) dv.slot_pos[phys] = s;
+      else phys = -1;
     }
     if (live) s_phys[i] = phys;
     if (fits) popped += total;
   }
-  if (tid == 0 && popped > 0) dv.ctrl[kCtrlFree] = fc - popped;
+  if (tid == 0 && popped > 0) *cs.free = fc - popped;
   __syncthreads();
 
   // ---- K and V rows into their slots: 16-byte vectors, consecutive threads
@@ -217,7 +224,8 @@ bulk_count_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     return;
   }
   const int st = seq * dv.hkv + kvh;
-  const int s0 = dv.pos[st];
+  const Cur cs = cur_state(dv, read_par(dv.ctrl));
+  const int s0 = cs.pos[st];
   int fresh = 0;
   for (int t = threadIdx.x; t < T; t += blockDim.x) {
     const int j = s0 + t;
@@ -225,14 +233,14 @@ bulk_count_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     if (j >= dv.w) {
       const int jp = j - dv.w;
       marked = (jp >= s0) ? alpha_at(asrc, (size_t)(t0 + jp - s0), kvh)
-                          : (dv.ring[(size_t)st * dv.w + jp % dv.w] & 1);
+                          : (dv.ring[ring_at(dv, st, jp)] & 1);
     }
     fresh += !marked;
   }
   int total;
   block_exclusive_scan(fresh, s_warp, &total);
   if (threadIdx.x == 0) {
-    const int n_final = dv.n[st] + total;
+    const int n_final = cs.n[st] + total;
     const int pages = (n_final + kPage - 1) / kPage;
     if (pages > dv.mps) {
       latch(dv.ctrl, DMS_ERR_STREAM_FULL);
@@ -255,7 +263,8 @@ bulk_pages_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids) {
   for (int i = b; i < e; ++i) cnt += dv.scratch[i];
   int total;
   int rank = block_exclusive_scan(cnt, s_warp, &total);
-  const int fc = dv.ctrl[kCtrlFree];
+  int32_t* free_depth = cur_state(dv, read_par(dv.ctrl)).free;
+  const int fc = *free_depth;
   if (total > fc) {
     if (threadIdx.x == 0) latch(dv.ctrl, DMS_ERR_POOL_EXHAUSTED);
     return;
@@ -266,12 +275,13 @@ bulk_pages_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids) {
     const int st = seq_ids[i / dv.hkv] * dv.hkv + i % dv.hkv;
     const int np0 = dv.n_pages[st];
     for (int q = 0; q < k; ++q)
-      dv.page_table[(size_t)st * dv.mps + np0 + q] = dv.free_list[fc - 1 - (rank + q)];
+      if (in_bounds(np0 + q, dv.mps, dv.ctrl) && in_bounds(fc - 1 - (rank + q), dv.max_pages, dv.ctrl))
+        dv.page_table[(size_t)st * dv.mps + np0 + q] = dv.free_list[fc - 1 - (rank + q)];
     rank += k;
     dv.n_pages[st] = np0 + k;
   }
   __syncthreads();
-  if (threadIdx.x == 0) dv.ctrl[kCtrlFree] = fc - total;
+  if (threadIdx.x == 0) *free_depth = fc - total;
 }
 
 // Bulk append, pass 3: slots, window ring, slot tags and rows, one block per
@@ -290,13 +300,13 @@ bulk_write_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
   const int bseq = i / dv.hkv, kvh = i % dv.hkv;
   const int st = seq_ids[bseq] * dv.hkv + kvh;
   const int t0 = cu[bseq], T = cu[bseq + 1] - t0;
-  const int s0 = dv.pos[st];
+  const Cur cs = cur_state(dv, read_par(dv.ctrl));
+  const int s0 = cs.pos[st];
   const int s_last = s0 + T - 1;
   const int row_bytes = dv.d * dv.elem_bytes;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   const int sub = min((int)blockDim.x, dv.w);
-  int n_cur = dv.n[st];
-  int32_t* ring = dv.ring + (size_t)st * dv.w;
+  int n_cur = cs.n[st];
   const int32_t* pt = dv.page_table + (size_t)st * dv.mps;
 
   for (int c0 = 0; c0 < T; c0 += sub) {
@@ -306,8 +316,8 @@ bulk_write_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     int r = 0;
     bool retire = false;
     if (active) {
-      r = ring[j % dv.w];
-      retire = (j >= dv.w) && (r & 1);
+      r = dv.ring[ring_leaving(dv, st, j)];   // token j - w (read before the scan's barrier,
+      retire = (j >= dv.w) && (r & 1);        // the new entries are written after it)
     }
     int total;
     const int pre = block_exclusive_scan(active && !retire ? 1 : 0, s_warp, &total);
@@ -315,14 +325,14 @@ bulk_write_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     if (active) {
       const int slot = retire ? (r >> 1) : n_cur + pre;
       const int a = alpha_at(asrc, (size_t)(t0 + t), kvh);
-      ring[j % dv.w] = (slot << 1) | a;
+      dv.ring[ring_at(dv, st, j)] = (slot << 1) | a;
       const bool dead = a && (j + dv.w <= s_last);
       const int page = slot / kPage < dv.mps ? pt[slot / kPage] : -1;
       if (page < 0 || page >= dv.max_pages) {
         latch(dv.ctrl, DMS_ERR_INVALID);
       } else if (!dead) {
         phys = page * kPage + slot % kPage;
-        dv.slot_pos[phys] = j;
+        dv.slot_pos[phys] = j;   // page checked above: phys < max_pages * 16
       }
     }
     if (tid < 256) s_phys[tid] = phys;
@@ -339,8 +349,8 @@ bulk_write_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
     __syncthreads();
   }
   if (tid == 0) {
-    dv.n[st] = n_cur;
-    dv.pos[st] = s0 + T;
+    cs.n[st] = n_cur;
+    cs.pos[st] = s0 + T;
   }
 }
 
@@ -350,6 +360,7 @@ bulk_write_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
 __global__ void __launch_bounds__(256) reset_seq_kernel(Dev dv, int seq) {
   __shared__ int s_off[kMaxKvHeads + 1];
   __shared__ int s_fc, s_ok;
+  const Cur cs = cur_state(dv, read_par(dv.ctrl));
   if (threadIdx.x == 0) {
     s_ok = read_status(dv.ctrl) == 0;
     int acc = 0;
@@ -358,7 +369,7 @@ __global__ void __launch_bounds__(256) reset_seq_kernel(Dev dv, int seq) {
       acc += dv.n_pages[seq * dv.hkv + k];
     }
     s_off[dv.hkv] = acc;
-    s_fc = dv.ctrl[kCtrlFree];
+    s_fc = *cs.free;
     if (s_ok && s_fc + acc > dv.max_pages) {
       latch(dv.ctrl, DMS_ERR_INVALID);
       s_ok = 0;
@@ -370,18 +381,19 @@ __global__ void __launch_bounds__(256) reset_seq_kernel(Dev dv, int seq) {
     const int st = seq * dv.hkv + k;
     const int np = s_off[k + 1] - s_off[k];
     for (int p = threadIdx.x; p < np; p += blockDim.x)
-      dv.free_list[s_fc + s_off[k] + (np - 1 - p)] = dv.page_table[(size_t)st * dv.mps + p];
-    for (int r = threadIdx.x; r < dv.w; r += blockDim.x) dv.ring[(size_t)st * dv.w + r] = 0;
+      if (in_bounds(s_fc + s_off[k] + (np - 1 - p), dv.max_pages, dv.ctrl) && in_bounds(p, dv.mps, dv.ctrl))
+        dv.free_list[s_fc + s_off[k] + (np - 1 - p)] = dv.page_table[(size_t)st * dv.mps + p];
+    for (int r = threadIdx.x; r <= dv.w; r += blockDim.x) dv.ring[(size_t)st * (dv.w + 1) + r] = 0;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     for (int k = 0; k < dv.hkv; ++k) {
       const int st = seq * dv.hkv + k;
-      dv.n[st] = 0;
-      dv.pos[st] = 0;
+      cs.n[st] = 0;
+      cs.pos[st] = 0;
       dv.n_pages[st] = 0;
     }
-    dv.ctrl[kCtrlFree] = s_fc + s_off[dv.hkv];
+    *cs.free = s_fc + s_off[dv.hkv];
   }
 }
 
@@ -391,17 +403,19 @@ __global__ void init_state_kernel(Dev dv) {
   const size_t nthr = (size_t)gridDim.x * blockDim.x;
   for (size_t k = tid; k < (size_t)dv.max_pages; k += nthr) dv.free_list[k] = dv.max_pages - 1 - (int)k;
   for (size_t k = tid; k < (size_t)dv.S; k += nthr) {
-    dv.pos[k] = 0;
-    dv.n[k] = 0;
     dv.n_pages[k] = 0;
     dv.scratch[k] = 0;
     dv.cnt[k] = 0;
   }
-  for (size_t k = tid; k < (size_t)dv.S * dv.w; k += nthr) dv.ring[k] = 0;
+  for (size_t k = tid; k < 2 * (size_t)dv.S; k += nthr) {   // both parities
+    dv.pos[k] = 0;
+    dv.n[k] = 0;
+  }
+  for (size_t k = tid; k < (size_t)dv.S * (dv.w + 1); k += nthr) dv.ring[k] = 0;
   if (tid == 0) {
-    dv.ctrl[kCtrlStatus] = 0;
+    for (int k = 0; k < kCtrlWords; ++k) dv.ctrl[k] = 0;   // status, parity 0, no step errors
     dv.ctrl[kCtrlFree] = dv.max_pages;
-    for (int k = 2; k < kCtrlWords; ++k) dv.ctrl[k] = 0;
+    dv.ctrl[kCtrlFree + 1] = dv.max_pages;
   }
 }
 
@@ -416,9 +430,10 @@ stats_kernel(Dev dv, int32_t* retained, int32_t* seen, float* head_cr, int64_t* 
   __shared__ unsigned long long s_head[kMaxKvHeads][2];
   for (int h = threadIdx.x; h < dv.hkv; h += blockDim.x) s_head[h][0] = s_head[h][1] = 0;
   grid_dependency_wait();
+  const Cur cs = cur_state(dv, read_par(dv.ctrl));
   __syncthreads();
   for (int st = threadIdx.x; st < dv.S; st += blockDim.x) {
-    const int r = dv.n[st], p = dv.pos[st];
+    const int r = cs.n[st], p = cs.pos[st];
     if (retained) retained[st] = r;
     if (seen) seen[st] = p;
     atomicAdd(&s_head[st % dv.hkv][0], (unsigned long long)p);
@@ -439,14 +454,23 @@ stats_kernel(Dev dv, int32_t* retained, int32_t* seen, float* head_cr, int64_t* 
   }
 }
 
+// Eviction decisions of `rows` tokens from the sign of a designated logit
+// channel: out[row][kvh] = alpha_at(src, row, kvh), one thread per decision.
+__global__ void __launch_bounds__(256) alpha_from_logit_kernel(AlphaSrc src, int rows, uint8_t* out) {
+  const size_t total = (size_t)rows * src.hkv;
+  for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < total; t += (size_t)gridDim.x * blockDim.x)
+    out[t] = (uint8_t)alpha_at(src, t / src.hkv, (int)(t % src.hkv));
+}
+
 // Gather the retained rows of one stream in logical slot order (warp per row).
 __global__ void __launch_bounds__(256)
 gather_kernel(Dev dv, int seq, int kvh, int rows_cap, uint8_t* Kout, uint8_t* Vout) {
   const int st = seq * dv.hkv + kvh;
-  const int rows = min(dv.n[st], rows_cap);
+  const int rows = min(cur_state(dv, read_par(dv.ctrl)).n[st], rows_cap);
   const int row_bytes = dv.d * dv.elem_bytes;
   const int lane = threadIdx.x & 31;
   for (int l = blockIdx.x * 8 + (threadIdx.x >> 5); l < rows; l += gridDim.x * 8) {
+    if (!in_bounds(l / kPage, dv.mps, dv.ctrl)) break;
     const int page = dv.page_table[(size_t)st * dv.mps + l / kPage];
     if (page < 0 || page >= dv.max_pages) continue;
     warp_copy_row(Kout + (size_t)l * row_bytes, page_row(dv, page, 0, l % kPage, row_bytes), row_bytes, lane);
@@ -465,7 +489,8 @@ cudaError_t prepare_aux_kernels() {
   const void* fns[] = {(const void*)append_decode_kernel, (const void*)bulk_count_kernel,
                        (const void*)bulk_pages_kernel, (const void*)bulk_write_kernel,
                        (const void*)reset_seq_kernel, (const void*)init_state_kernel,
-                       (const void*)stats_kernel, (const void*)gather_kernel};
+                       (const void*)stats_kernel, (const void*)gather_kernel,
+                       (const void*)alpha_from_logit_kernel};
   for (const void* f : fns) {
     cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                          (int)cudaSharedmemCarveoutMaxShared);
@@ -508,9 +533,7 @@ cudaError_t launch_init_state(const Dev& dv, cudaStream_t st) {
 }
 
 cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
-                                 const void* K, const void* V, const uint8_t* alpha, int alpha_channel,
-                                 int* launches) {
-  const AlphaSrc asrc{alpha, (const uint8_t*)K, alpha_channel, dv.hkv, dv.d, dv.elem_bytes};
+                                 const void* K, const void* V, const AlphaSrc& asrc, int* launches) {
   const int nst = n_seqs * dv.hkv;
   if (nst == 0) return cudaSuccess;
   *launches += 1;
@@ -520,8 +543,7 @@ cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, con
 
 cudaError_t launch_append_bulk(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
                                const int32_t* cu_tokens, int total_tokens, const void* K, const void* V,
-                               const uint8_t* alpha, int alpha_channel, int* launches) {
-  const AlphaSrc asrc{alpha, (const uint8_t*)K, alpha_channel, dv.hkv, dv.d, dv.elem_bytes};
+                               const AlphaSrc& asrc, int* launches) {
   const int nst = n_seqs * dv.hkv;
   if (nst == 0) return cudaSuccess;
   bulk_count_kernel<<<nst, 256, 0, st>>>(dv, n_seqs, seq_ids, cu_tokens, total_tokens, asrc);
@@ -540,6 +562,14 @@ cudaError_t launch_reset_seq(const Dev& dv, cudaStream_t st, int seq) {
 cudaError_t launch_stats(const Dev& dv, cudaStream_t st, int32_t* retained, int32_t* seen, float* head_cr,
                          int64_t* totals) {
   return launch_dependent(stats_kernel, dim3(1), dim3(256), 0, st, dv, retained, seen, head_cr, totals);
+}
+
+cudaError_t launch_alpha_from_logit(cudaStream_t st, const AlphaSrc& src, int rows, uint8_t* out) {
+  const size_t total = (size_t)rows * src.hkv;
+  if (total == 0) return cudaSuccess;
+  const int blocks = (int)std::min<size_t>((total + 255) / 256, 4096);
+  alpha_from_logit_kernel<<<blocks, 256, 0, st>>>(src, rows, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gather(const Dev& dv, cudaStream_t st, int seq, int kvh, int rows_cap, void* Kout,

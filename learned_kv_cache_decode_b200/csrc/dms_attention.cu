@@ -46,6 +46,14 @@ namespace dms {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+// Stages per warp filled before the dependency wait of an early start; the
+// rest of a warp's first `spw` pages go out right after the round trip that
+// checks the guess has been issued, so that round trip is not queued behind
+// the whole first burst of page copies.
+#ifndef DMS_PRE_STAGES
+#define DMS_PRE_STAGES 8
+#endif
+constexpr int kPreStages = DMS_PRE_STAGES;
 constexpr int kRslotUnknown = -2;   // leaving slot not known until the window ring is read
 
 // A decode step fused into the attention launch: the new token of every call
@@ -54,7 +62,6 @@ struct StepArgs {
   const uint8_t* K;       // [n_seqs][hkv][d] new key rows
   const uint8_t* V;       // [n_seqs][hkv][d] new value rows
   AlphaSrc asrc;          // eviction decisions of the new tokens
-  unsigned long long launch_index;   // fused steps launched on this cache before this one
   Dev dv;                 // the cache, writable
   NextPlan next;          // schedule left by the previous fused step, and the one this step leaves
   unsigned long long trust;   // tag of the schedule to read (0: none, plan from the cache state)
@@ -66,13 +73,16 @@ struct AttnArgs {
   const int32_t* seq_ids;
   const uint8_t* Q;
   uint8_t* out;
-  const int32_t* n;
+  const int32_t* n;       // retained counts: n + par * n_stride is the current copy
   const int32_t* page_table;
   const uint8_t* kv;
   int32_t* ctrl;
   float* part;
   int32_t* cnt;
+  int part_slots;   // partial slots in `part` (debug-build bounds)
   int n_seqs, hkv, g, hq, mps, max_seqs, max_pages, out_f32;
+  int n_stride;   // elements between the two parity copies of the counts (0: one copy)
+  int par;        // state parity (fused step: before the step); < 0: read the cache's parity word
   float sl2e;   // softmax scale * log2(e): scores live in the base-2 domain
   int spw;      // TMA stages per warp
   int S;        // streams of the cache (sizes the plan arrays in shared memory)
@@ -83,6 +93,19 @@ struct AttnArgs {
   int32_t* guess_wr;
   int pre_attn;
 };
+
+// A retained count as the kernel uses it: clamped to what a stream's page
+// table can address, [0, 16 * mps]. Counts the library keeps are always in
+// range; caller-owned counts (the allocation-free entry point) are checked here,
+// and an out-of-range one latches DMS_ERR_INVALID.
+__device__ __forceinline__ int clamp_count(int n, int mps, int32_t* ctrl) {
+  const int hi = kPage * mps;
+  if (n < 0 || n > hi) {
+    latch(ctrl, DMS_ERR_INVALID);
+    n = n < 0 ? 0 : hi;
+  }
+  return n;
+}
 
 // Largest i in [0, n] with prefix[i] <= x (prefix is non-decreasing, prefix[0] = 0).
 __device__ __forceinline__ int stream_of(const int* prefix, int n, int x) {
@@ -514,6 +537,7 @@ __device__ __forceinline__ void combine_stream(const AttnArgs& a, int i, int fir
   const int b = i / a.hkv, kvh = i % a.hkv;
   const int items = a.g * (D / 4);
   const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
+  if (!in_bounds((long long)last + i, a.part_slots, a.ctrl)) last = first - 1;   // (debug build)
   for (int t0 = 0; t0 < items; t0 += t_step) {
     const int t = t0 + t_begin;
     const bool live = t < items;
@@ -547,23 +571,31 @@ __device__ __forceinline__ void combine_stream(const AttnArgs& a, int i, int fir
 //  1. For every call stream, from the pre-step state read by the plan and the
 //     leaving slot the consumer warps read from the window ring: does the
 //     token at s - w leave now (its slot is reused), or does the new token
-//     take the fresh slot n (popping a page when n is a multiple of 16)? Pops are ranked in stream order (warp scan), exactly
-//     as dms_append ranks them; a pool too small for all pops fails every
-//     stream that needs one.
-//  2. Publishes the decisions to the CTA's consumers, then counts this CTA as
-//     having read the pre-step state.
-//  3. Writes the outputs of this CTA's streams that had nothing retained (the
+//     take the fresh slot n (popping a page when n is a multiple of 16)? Pops
+//     are ranked in stream order (warp scan), exactly as dms_append ranks them;
+//     a pool too small for all pops fails every stream that needs one.
+//  2. Publishes the decisions to the CTA's consumers.
+//  3. Writes the state of the next parity that falls to this CTA: the counts of
+//     its share of the streams the call does not append to, copied over, and
+//     (CTA 0) the parity word and the free-stack depth.
+//  4. Writes the outputs of this CTA's streams that had nothing retained (the
 //     new token alone: its value row).
-//  4. Once every CTA has read the pre-step state, appends this CTA's streams
-//     (i = blockIdx.x mod gridDim.x): bookkeeping and K/V rows. CTA 0 latches
-//     the errors the plan found and moves the free stack.
+//  5. Appends this CTA's call streams (i = blockIdx.x mod gridDim.x):
+//     bookkeeping into the next parity and the window ring, and the K/V rows.
+// Nothing here waits on another CTA: every word it writes is one that no CTA
+// of this launch reads (the other parity's counts, the ring entry of token s
+// rather than that of s - w, page-table entries past the pre-step pages, rows
+// the attention masks or that lie past the pre-step counts).
 template <int D, typename E>
 __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int* prefix, const int* sid,
                                        const int* s_nold, const int* s_pos, int* s_rslot, int* s_tslot,
-                                       int* s_flag, int* s_rank, int* misc, bool healthy,
+                                       int* s_flag, int* s_rank, int* misc, uint32_t* bits, bool healthy,
                                        volatile int* abort_flag, int K0, int K1) {
   const int lane = threadIdx.x & 31;
   const Dev& dv = a.step.dv;
+  const int G = gridDim.x;
+  const int par = a.par, nxt = par ^ 1;
+  const Cur rd = cur_state(dv, par), wr = cur_state(dv, nxt);
   // Wait (no spinning) until the consumer warps have resolved every stream's
   // leaving slot (s_rslot): they arrive at barrier 2 without waiting.
   named_barrier(2, blockDim.x);
@@ -615,9 +647,49 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
   if (lane == 0) {
     __threadfence_block();
     *reinterpret_cast<volatile int*>(&misc[15]) = 1;   // the consumers may read the decisions
-    // This CTA is done reading the pre-step state (its reads were ordered
-    // before this point by the plan's barriers and barrier 2).
-    red_add_release_gpu_u64(reinterpret_cast<unsigned long long*>(&a.ctrl[kCtrlPlanned]), 1ull);
+  }
+
+  // The counts of the next parity. A stream the call appends to is written by
+  // the CTA that appends it (below); this CTA copies over its share (stream id
+  // = blockIdx.x mod gridDim.x) of the others, or of every stream when the
+  // cache is poisoned and nothing is appended.
+  const int words = (dv.S + 31) / 32;
+  for (int k = lane; k < words; k += 32) bits[k] = 0u;
+  __syncwarp();
+  if (healthy)
+    for (int i = lane; i < nst; i += 32)
+      if (!(s_flag[i] & 4)) atomicOr(&bits[sid[i] >> 5], 1u << (sid[i] & 31));
+  __syncwarp();
+  for (int st = blockIdx.x + G * lane; st < dv.S; st += G * 32) {
+    if (healthy && ((bits[st >> 5] >> (st & 31)) & 1u)) continue;
+    wr.n[st] = rd.n[st];
+    wr.pos[st] = rd.pos[st];
+  }
+  if (blockIdx.x == 0) {
+    // The error of the first call stream that has one (bad seq id before stream
+    // full before pool exhausted), found by the whole warp.
+    int first = 0x7fffffff;
+    if (healthy)
+      for (int i = lane; i < nst; i += 32)
+        if (s_flag[i] & (4 | 8 | 16)) {
+          first = i;
+          break;
+        }
+    first = __reduce_min_sync(0xffffffffu, first);
+    if (lane == 0) {
+      dv.ctrl[kCtrlPar] = nxt;   // read by the kernels that run after this launch
+      if (healthy) {
+        if (first < nst) {
+          const int f = s_flag[first];
+          latch_word(dv.ctrl + kCtrlStepErr + nxt,
+                     (f & 4) ? DMS_ERR_BAD_SEQ : (f & 8) ? DMS_ERR_STREAM_FULL : DMS_ERR_POOL_EXHAUSTED);
+        }
+        *wr.free = misc[13] > 0 ? misc[12] - misc[13] : misc[12];
+      } else {
+        *wr.free = misc[12];
+        latch_word(dv.ctrl + kCtrlStepErr + nxt, misc[16]);   // the error stays visible to the next step
+      }
+    }
   }
   __syncwarp();
   if (!healthy) return;
@@ -645,7 +717,6 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
     k = pe;
   }
 
-  const int G = gridDim.x;
   // Streams with nothing retained before the step attend to the new token alone.
   for (int i = blockIdx.x; i < nst; i += G) {
     if (prefix[i + 1] != prefix[i]) continue;
@@ -666,127 +737,181 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
   // come from the page table (this step writes only entries past them), a
   // popped one from the free stack (never written by a step). Nothing reads
   // this buffer during this launch: it is the one of the other tag parity.
-  // Eight loads per lane are in flight at a time.
+  // Eight loads per lane are in flight at a time; the first batch's loads go
+  // out together with those of the appends below.
+  const int wbuf = (int)(a.step.wtag & 1ull);
+  long long c0 = 0, c1 = 0;
+  int32_t* lst = nullptr;
+  size_t cell = 0;
   if (a.step.next.entry != nullptr && misc[13] >= 0) {
     const long long P2 = (long long)prefix[nst] + misc[13];
     const long long Ge = P2 < G ? P2 : G;
-    const long long c0 = blockIdx.x < Ge ? blockIdx.x * P2 / Ge : 0;
-    const long long c1 = blockIdx.x < Ge ? (blockIdx.x + 1) * P2 / Ge : 0;
+    c0 = blockIdx.x < Ge ? blockIdx.x * P2 / Ge : 0;
+    c1 = blockIdx.x < Ge ? (blockIdx.x + 1) * P2 / Ge : 0;
     if (c1 - c0 <= a.step.next.cap) {
-      const size_t cell = (size_t)(a.step.wtag & 1ull) * G + blockIdx.x;
-      int32_t* lst = a.step.next.list + cell * a.step.next.cap;
-      const int fc = misc[12];
-      for (long long base = c0; base < c1; base += 32 * 8) {
-        int v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const long long kk = base + lane + 32 * u;
-          v[u] = 0;
-          if (kk < c1) {
-            int lo = 0, hi = nst;   // largest i with prefix[i] + s_rank[i] <= kk
-            while (hi - lo > 1) {
-              const int mid = (lo + hi) >> 1;
-              if (prefix[mid] + s_rank[mid] <= kk) lo = mid; else hi = mid;
-            }
-            const int p = (int)(kk - prefix[lo] - s_rank[lo]);
-            v[u] = p < prefix[lo + 1] - prefix[lo] ? __ldg(dv.page_table + (size_t)sid[lo] * dv.mps + p)
-                                                   : __ldg(dv.free_list + (fc - 1 - s_rank[lo]));
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const long long kk = base + lane + 32 * u;
-          if (kk < c1) lst[kk - c0] = v[u];
-        }
-      }
-      __syncwarp();
+      cell = (size_t)wbuf * G + blockIdx.x;
+      lst = a.step.next.list + cell * a.step.next.cap;
       if (lane == 0) {
         a.step.next.hdr[2 * cell] = make_int4((int)(uint32_t)a.step.wtag, (int)(uint32_t)(a.step.wtag >> 32), nst, (int)P2);
         a.step.next.hdr[2 * cell + 1] = make_int4((int)c0, (int)c1, 0, 0);
       }
     }
   }
-  // The window-ring entry the next step reads for this CTA's first stream
-  // (residue s + 1, which this step does not write when w > 1), requested now.
-  int rn_first = 0;
-  if (a.step.next.entry != nullptr && lane == 0 && blockIdx.x < nst && dv.w > 1 && s_tslot[blockIdx.x] >= 0)
-    rn_first = dv.ring[(size_t)sid[blockIdx.x] * dv.w + ((s_pos[blockIdx.x] + 1) % dv.w)];
-
-  // Wait until every CTA has read the pre-step state, then write the append.
-  if (lane == 0) {
-    // Every launch adds one per CTA, and the grid is the same for every
-    // launch on this cache: this launch is complete at (index + 1) * grid.
-    wait_count_ge(reinterpret_cast<const volatile unsigned long long*>(&a.ctrl[kCtrlPlanned]),
-                  (a.step.launch_index + 1ull) * (unsigned long long)G, abort_flag, a.ctrl, 200);
-    fence_acq_rel_gpu();   // acquire: every CTA's reads of the pre-step state happen before our writes
-  }
-  __syncwarp();
-  if (blockIdx.x == 0 && lane == 0) {
-    for (int i = 0; i < nst; ++i) {
-      const int f = s_flag[i];
-      if (f & 4) latch(a.ctrl, DMS_ERR_BAD_SEQ);
-      if (f & 8) latch(a.ctrl, DMS_ERR_STREAM_FULL);
-      if (f & 16) latch(a.ctrl, DMS_ERR_POOL_EXHAUSTED);
+  const int fc = misc[12];
+  // Page id of position kk of the next step's concatenated order (kk < c1).
+  auto list_page = [&](long long kk) -> int {
+    int lo = 0, hi = nst;   // largest i with prefix[i] + s_rank[i] <= kk
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (prefix[mid] + s_rank[mid] <= kk) lo = mid; else hi = mid;
     }
-    if (misc[13] > 0) dv.ctrl[kCtrlFree] = misc[12] - misc[13];
+    const int p = (int)(kk - prefix[lo] - s_rank[lo]);
+    if (p < prefix[lo + 1] - prefix[lo]) {
+      if (in_bounds(sid[lo], dv.S, a.ctrl) && in_bounds(p, dv.mps, a.ctrl))
+        return __ldg(dv.page_table + (size_t)sid[lo] * dv.mps + p);
+    } else if (in_bounds(fc - 1 - s_rank[lo], dv.max_pages, a.ctrl)) {
+      return __ldg(dv.free_list + (fc - 1 - s_rank[lo]));
+    }
+    return 0;
+  };
+  int lv0 = 0, lv1 = 0, lv2 = 0, lv3 = 0, lv4 = 0, lv5 = 0, lv6 = 0, lv7 = 0;   // first batch, in registers
+  if (lst != nullptr) {
+    if (c0 + lane < c1) lv0 = list_page(c0 + lane);
+    if (c0 + lane + 32 < c1) lv1 = list_page(c0 + lane + 32);
+    if (c0 + lane + 64 < c1) lv2 = list_page(c0 + lane + 64);
+    if (c0 + lane + 96 < c1) lv3 = list_page(c0 + lane + 96);
+    if (c0 + lane + 128 < c1) lv4 = list_page(c0 + lane + 128);
+    if (c0 + lane + 160 < c1) lv5 = list_page(c0 + lane + 160);
+    if (c0 + lane + 192 < c1) lv6 = list_page(c0 + lane + 192);
+    if (c0 + lane + 224 < c1) lv7 = list_page(c0 + lane + 224);
   }
-  const int row_bytes = D * (int)sizeof(E);
-  const int vec = row_bytes / 16;
+
+  // Append this CTA's call streams: bookkeeping into the next parity and the
+  // window ring (the entry of token s, never the one of s - w that the plan
+  // reads), the K/V rows into a masked row or one past the pre-step count. A
+  // stream left unchanged (stream full, pool exhausted) carries its counts over.
+  // Every load of one stream's append (its page id, the ring entry for the next
+  // step's schedule, the new K and V rows) is issued before any store: one
+  // memory round trip per stream, which the page stream of the consumers keeps
+  // long.
+  constexpr int kRowBytes = D * (int)sizeof(E);
+  constexpr int kVec = kRowBytes / 16;                  // 16-byte vectors per row
+  constexpr int kPerLane = (2 * kVec + 31) / 32;        // K and V vectors per lane
+  PlanEntry* entries = a.step.next.entry != nullptr ? a.step.next.entry + (size_t)wbuf * a.step.next.S : nullptr;
   for (int i = blockIdx.x; i < nst; i += G) {
     const int ts = s_tslot[i];
-    if (ts < 0) continue;
     const int st = sid[i], s = s_pos[i], f = s_flag[i];
-    const int lp = ts / kPage;
-    const int page = (f & 1) ? dv.free_list[misc[12] - 1 - s_rank[i]] : dv.page_table[(size_t)st * dv.mps + lp];
+    if (f & 4) continue;   // bad seq id: no stream
+    int page = -1, rn = 0;
+    uint4 x[kPerLane];
+    if (ts >= 0) {
+      if (lane == 0) {
+        if (f & 1) {
+          if (in_bounds(fc - 1 - s_rank[i], dv.max_pages, a.ctrl)) page = dv.free_list[fc - 1 - s_rank[i]];
+        } else if (in_bounds(st, dv.S, a.ctrl) && in_bounds(ts / kPage, dv.mps, a.ctrl)) {
+          page = dv.page_table[(size_t)st * dv.mps + ts / kPage];
+        }
+      }
+      if (lane == 1 && entries != nullptr && dv.w > 1) rn = dv.ring[ring_leaving(dv, st, s + 1)];
+#pragma unroll
+      for (int c = 0; c < kPerLane; ++c) {
+        const int v = lane + 32 * c;
+        if (v < 2 * kVec)
+          x[c] = __ldg(reinterpret_cast<const uint4*>((v >= kVec ? a.step.V : a.step.K) + (size_t)i * kRowBytes) +
+                       (v % kVec));
+      }
+    }
+    page = __shfl_sync(0xffffffffu, page, 0);
+    rn = __shfl_sync(0xffffffffu, rn, 1);
     if (page < 0 || page >= dv.max_pages) {
-      if (lane == 0) latch(a.ctrl, DMS_ERR_INVALID);
+      if (lane == 0) {
+        if (ts >= 0) latch(a.ctrl, DMS_ERR_INVALID);
+        wr.n[st] = s_nold[i];
+        wr.pos[st] = s;
+      }
       continue;
     }
     if (lane == 0) {
+      const int lp = ts / kPage;
       const int nnew = s_rslot[i] < 0 ? s_nold[i] + 1 : s_nold[i];
       const int rent = (ts << 1) | ((f >> 1) & 1);
-      if (f & 1) {
+      if ((f & 1) && in_bounds(lp, dv.mps, a.ctrl)) {
         dv.page_table[(size_t)st * dv.mps + lp] = page;
         dv.n_pages[st] = lp + 1;
       }
-      if (s_rslot[i] < 0) dv.n[st] = nnew;
-      dv.ring[(size_t)st * dv.w + (s % dv.w)] = rent;
-      dv.pos[st] = s + 1;
+      wr.n[st] = nnew;
+      wr.pos[st] = s + 1;
+      dv.ring[ring_at(dv, st, s)] = rent;
       dv.slot_pos[(size_t)page * kPage + ts % kPage] = s;
-      if (a.step.next.entry != nullptr) {
-        // The schedule entry of call stream i for the next step. Its window-ring
-        // entry is the one at residue s + 1: the one just written when w = 1,
-        // else one this step leaves alone.
-        const int rnext = dv.w == 1 ? rent
-                          : (i == (int)blockIdx.x ? rn_first : dv.ring[(size_t)st * dv.w + ((s + 1) % dv.w)]);
-        PlanEntry* e = a.step.next.entry + i;
-        *reinterpret_cast<int4*>(e) = make_int4(nnew, s + 1, rnext, st / a.hkv);
+      if (entries != nullptr) {
+        // The schedule entry of call stream i for the next step: the ring entry
+        // of the token that leaves then (s + 1 - w), the one just written when
+        // w = 1, else one this step leaves alone.
+        PlanEntry* e = entries + i;
+        *reinterpret_cast<int4*>(e) = make_int4(nnew, s + 1, dv.w == 1 ? rent : rn, st / a.hkv);
         e->tag = a.step.wtag;
         e->first = prefix[i] + s_rank[i];
       }
     }
-    for (int v = lane; v < 2 * vec; v += 32) {
-      const int which = v / vec, c = v % vec;
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>((which ? a.step.V : a.step.K) + (size_t)i * row_bytes) + c);
-      reinterpret_cast<uint4*>(dv.kv + ((size_t)page * 2 * kPage + (size_t)which * kPage + ts % kPage) * row_bytes)[c] = x;
+#pragma unroll
+    for (int c = 0; c < kPerLane; ++c) {
+      const int v = lane + 32 * c;
+      if (v < 2 * kVec) {
+        const int which = v >= kVec;
+        reinterpret_cast<uint4*>(dv.kv + ((size_t)page * 2 * kPage + (size_t)which * kPage + ts % kPage) * kRowBytes)
+            [v % kVec] = x[c];
+      }
+    }
+  }
+
+  if (lst != nullptr) {
+    const long long l0 = lane;
+    if (c0 + l0 < c1) lst[l0] = lv0;
+    if (c0 + l0 + 32 < c1) lst[l0 + 32] = lv1;
+    if (c0 + l0 + 64 < c1) lst[l0 + 64] = lv2;
+    if (c0 + l0 + 96 < c1) lst[l0 + 96] = lv3;
+    if (c0 + l0 + 128 < c1) lst[l0 + 128] = lv4;
+    if (c0 + l0 + 160 < c1) lst[l0 + 160] = lv5;
+    if (c0 + l0 + 192 < c1) lst[l0 + 192] = lv6;
+    if (c0 + l0 + 224 < c1) lst[l0 + 224] = lv7;
+    for (long long base = c0 + 32 * 8; base < c1; base += 32 * 8) {   // longer ranges: 8 loads in flight per lane
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = base + lane + 32 * u < c1 ? list_page(base + lane + 32 * u) : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (base + lane + 32 * u < c1) lst[base + lane + 32 * u - c0] = v[u];
     }
   }
 
   // The stream of the range's last piece, when other CTAs hold pieces of it:
-  // if they have all published theirs by now (they are usually done long
-  // before this CTA reaches the end of its range), the consumers will be the
-  // last to finish the stream and can combine without publishing their own
-  // piece and taking a ticket. The acquire read makes the other pieces'
-  // partials visible to them (CTA fence, then the flag).
+  // if they have all published theirs by the time the consumers start that
+  // piece (they usually are: the next CTA finishes the stream's tail at the
+  // start of its range), the consumers will be the last to finish the stream
+  // and can combine without publishing their own piece and taking a ticket.
+  // The acquire read makes the other pieces' partials visible to them (CTA
+  // fence, then the flag). The wait for the consumers is bounded; giving up
+  // only skips the shortcut.
   if (lane == 0 && K1 > K0) {
     const int il = stream_of(prefix, nst, K1 - 1);
     if (prefix[il] < K0 || prefix[il + 1] > K1) {
-      const long long P = prefix[nst];
-      const long long Geff = P < G ? P : G;
-      const int first = range_of(prefix[il], P, Geff), last = range_of(prefix[il + 1] - 1, P, Geff);
-      const bool done = ld_acquire_gpu(&a.cnt[il]) == last - first;
-      __threadfence_block();
-      *reinterpret_cast<volatile int*>(&misc[3]) = done ? 1 : 2;
+      const long long t0 = clock64();
+      bool started = true;
+      while (*reinterpret_cast<volatile int*>(&misc[17]) == 0) {
+        __nanosleep(256);
+        if (*abort_flag || clock64() - t0 > (1ll << 31)) {
+          started = false;
+          break;
+        }
+      }
+      if (started) {
+        const long long P = prefix[nst];
+        const long long Geff = P < G ? P : G;
+        const int first = range_of(prefix[il], P, Geff), last = range_of(prefix[il + 1] - 1, P, Geff);
+        const bool done = ld_acquire_gpu(&a.cnt[il]) == last - first;
+        __threadfence_block();
+        *reinterpret_cast<volatile int*>(&misc[3]) = done ? 1 : 2;
+      }
     }
   }
 }
@@ -811,7 +936,7 @@ __device__ __forceinline__ void issue_page(uint64_t* myfull, uint8_t* mystage, i
 
 // Shared-memory layout of one CTA (byte offsets from a 1024-aligned base).
 struct SmemLayout {
-  int stages, bars, misc, merge, prefix, sid, step, total;
+  int stages, bars, misc, merge, prefix, sid, step, bits, total;
 };
 
 __host__ __device__ inline SmemLayout smem_layout(int ncw, int spw, int stage_bytes, int d, int S, bool step) {
@@ -819,11 +944,12 @@ __host__ __device__ inline SmemLayout smem_layout(int ncw, int spw, int stage_by
   L.stages = 0;
   L.bars = ncw * spw * stage_bytes;
   L.misc = L.bars + 8 * ncw * spw;
-  L.merge = L.misc + 64;
+  L.merge = L.misc + 128;
   L.prefix = L.merge + ncw * kMaxGroup * (d + 2) * 4;
   L.sid = L.prefix + (S + 1) * 4;
   L.step = L.sid + S * 4;
-  L.total = L.step + (step ? 6 * S * 4 : 0);   // per-stream step decisions
+  L.bits = L.step + (step ? 6 * S * 4 : 0);               // per-stream step decisions
+  L.total = L.bits + (step ? ((S + 31) / 32) * 4 : 0);   // the call's streams, one bit per cache stream
   return L;
 }
 
@@ -874,8 +1000,10 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   // [3] the other pieces of the range's last stream are all published (1) or not (2), [4] the
   // consumers' snapshot of [3]), [12] free-stack depth
   // and [13] pages popped by this step (-1: pool exhausted), [14] stream whose combine a split
-  // first piece left to the end of the range (-1: none), [15] step decisions ready
+  // first piece left to the end of the range (-1: none), [15] step decisions ready, [16] the
+  // status word the plan read, [17] STEP: the consumers have started the range's last piece
   int* misc = reinterpret_cast<int*>(smem + lay.misc);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + lay.bits);
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(smem + lay.merge);
   int* prefix = reinterpret_cast<int*>(smem + lay.prefix);
   int* sid = reinterpret_cast<int*>(smem + lay.sid);
@@ -893,15 +1021,32 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nst = a.n_seqs * a.hkv;
   volatile int* abort_flag = misc;
+  // The status this launch acts on. A fused step of parity p reads the common
+  // word and the step-error word of parity p (errors it finds itself go to the
+  // other one); every other launch reads all of them.
+  auto launch_status = [&]() -> int {
+    if constexpr (STEP) {
+      const int s0 = read_word(&a.ctrl[kCtrlStatus]);
+      const int e = read_word(&a.ctrl[kCtrlStepErr + a.par]);
+      return s0 != 0 ? s0 : e;
+    } else {
+      return read_status(a.ctrl);
+    }
+  };
 
   if (tid == 0) {
     if constexpr (MMA) prefetch_tensormap(&tmap);
     misc[0] = 0;
     misc[14] = -1;
     misc[15] = 0;
+    misc[17] = 0;
     for (int s = 0; s < NCW * spw; ++s) mbar_init(smem_addr(&full[s]), 1);
     fence_mbar_init();
   }
+  // The state parity the counts are read at: the host's, or (attention launched
+  // into a stream under capture, a.par < 0) the cache's parity word, read with
+  // the seq ids in the plan.
+  int cpar = a.par;
   // Call streams [b0, e0) of this thread in the plan.
   const int per = (nst + kThreads - 1) / kThreads;
   const int b0 = min(tid * per, nst), e0 = min(b0 + per, nst);
@@ -946,18 +1091,19 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     if constexpr (MMA) mma_fetch_q<D>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
     else simt_fetch_q<D, E>(qcur, a, stream / a.hkv, stream % a.hkv, lane);
   };
+  const PlanEntry* tentries = STEP ? a.step.next.entry + (size_t)tbuf * a.step.next.S : nullptr;
   if (STEP && trust != 0 && a.step.pre != 0) {
     load_schedule_head();
     const int4 trange = ld_early4(a.step.next.hdr + 2 * ((size_t)tbuf * gridDim.x + blockIdx.x) + 1);
-    const int status = tid == 0 ? read_status(a.ctrl) : 0;
-    const int free_depth = tid == 0 ? *reinterpret_cast<const volatile int32_t*>(&a.ctrl[kCtrlFree]) : 0;
+    const int status = tid == 0 ? launch_status() : 0;
+    const int free_depth = tid == 0 ? read_word(&a.ctrl[kCtrlFree + a.par]) : 0;
     bool miss = false;
     for (int i = b0; i < e0; ++i) {
-      const int4 en = ld_early4(reinterpret_cast<const int4*>(a.step.next.entry + i));
-      const int4 e2 = ld_early4(reinterpret_cast<const int4*>(a.step.next.entry + i) + 1);   // tag, first
+      const int4 en = ld_early4(reinterpret_cast<const int4*>(tentries + i));
+      const int4 e2 = ld_early4(reinterpret_cast<const int4*>(tentries + i) + 1);   // tag, first
       const unsigned long long etag = (unsigned long long)(uint32_t)e2.x | ((unsigned long long)(uint32_t)e2.y << 32);
       const bool ok = etag == trust && en.w >= 0 && en.w < a.max_seqs;
-      const int nn = ok ? en.x : 0;
+      const int nn = ok ? clamp_count(en.x, a.mps, a.ctrl) : 0;
       s_nold[i] = nn;
       s_pos[i] = en.y;
       s_flag[i] = 0;
@@ -972,6 +1118,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       prefix[0] = 0;
       misc[1] = (status == 0);
       misc[12] = free_depth;
+      misc[16] = status;
     }
     any_miss = __syncthreads_or(miss) != 0;
     const long long P0 = prefix[nst];
@@ -981,7 +1128,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     pre_k1 = k1;
     if (pre_ok && warp < NCW) {
       const int nj = k1 - k0 > warp ? (k1 - k0 - warp + NCW - 1) / NCW : 0;
-      for (int j = 0; j < spw && j < nj; ++j) {
+      for (int j = 0; j < spw && j < kPreStages && j < nj; ++j) {
         int pg = __shfl_sync(0xffffffffu, spec_pg, j);
         if (lane == 0) {
           if (pg < 0 || pg >= a.max_pages) {
@@ -1001,7 +1148,8 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   // and the pages are cache state, final before the wait when the kernel before
   // this one does not write this cache. The guess is checked after the wait.
   int pid_pre = 0;   // consumer lanes: page id of the warp's job `lane` in the guessed plan
-  if (!STEP && a.pre_attn) {
+  if (!STEP && a.pre_attn) {   // (taken only when the host knows the parity: a.par >= 0)
+    const int32_t* ncur = a.n + (size_t)cpar * a.n_stride;
     const int status = tid == 0 ? read_status(a.ctrl) : 0;
     const int gcount = ld_early(a.guess_rd);
     bool bad = false;
@@ -1013,7 +1161,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
         bad = true;
       } else {
         st = seq * a.hkv + i % a.hkv;
-        pages = (ld_early(a.n + st) + kPage - 1) / kPage;   // through L2: written by earlier launches
+        pages = (clamp_count(ld_early(ncur + st), a.mps, a.ctrl) + kPage - 1) / kPage;   // through L2
       }
       sid[i] = st;
       prefix[i + 1] = pages;
@@ -1041,13 +1189,14 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
         if (lane < nj) {
           const int kk = pre_k0 + warp + NCW * lane;
           const int i = stream_of(prefix, nst, kk);
-          pid_pre = ld_early(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i]));
+          if (in_bounds(sid[i], (long long)a.max_seqs * a.hkv, a.ctrl) && in_bounds(kk - prefix[i], a.mps, a.ctrl))
+            pid_pre = ld_early(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i]));
           if (pid_pre < 0 || pid_pre >= a.max_pages) {
             latch(a.ctrl, DMS_ERR_INVALID);
             pid_pre = 0;
           }
         }
-        for (int j = 0; j < spw && j < nj; ++j) {
+        for (int j = 0; j < spw && j < kPreStages && j < nj; ++j) {
           const int pg = __shfl_sync(0xffffffffu, pid_pre, j);
           if (lane == 0)
             issue_page<D, MMA, E>(full + warp * spw, smem + lay.stages + (size_t)warp * spw * kStage, spw, j, pg,
@@ -1066,8 +1215,40 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     // The call's seq ids against the guess, and (STEP) the alpha of its new
     // tokens, in the same round trip as the query of the CTA's first piece.
     if (warp < NCW && pre_k1 > pre_k0) fetch_query(stream_of(prefix, nst, pre_k0));
+    // The first streams' seq ids (and alpha) are requested before the rest of
+    // the pre-planned copies, their values used after.
+    constexpr int kFirst = 4;
+    int seqv[kFirst], alv[kFirst];
+#pragma unroll
+    for (int u = 0; u < kFirst; ++u) {
+      const int i = b0 + u;
+      seqv[u] = i < e0 ? a.seq_ids[i / a.hkv] : 0;
+      alv[u] = (STEP && i < e0) ? alpha_at(a.step.asrc, (size_t)(i / a.hkv), i % a.hkv) : 0;
+    }
+    if (kPreStages < spw && warp < NCW) {   // warp-collective (page ids shuffled from the lanes)
+      const int nj = pre_k1 - pre_k0 > warp ? (pre_k1 - pre_k0 - warp + NCW - 1) / NCW : 0;
+      for (int j = kPreStages; j < spw && j < nj; ++j) {
+        int pg = __shfl_sync(0xffffffffu, STEP ? spec_pg : pid_pre, j);
+        if (lane == 0) {
+          if (pg < 0 || pg >= a.max_pages) {
+            latch(a.ctrl, DMS_ERR_INVALID);
+            pg = 0;
+          }
+          issue_page<D, MMA, E>(full + warp * spw, smem + lay.stages + (size_t)warp * spw * kStage, spw, j, pg,
+                                &tmap, a.kv);
+        }
+      }
+    }
     bool bad = false;
-    for (int i = b0; i < e0; ++i) {
+#pragma unroll
+    for (int u = 0; u < kFirst; ++u) {
+      const int i = b0 + u;
+      if (i < e0) {
+        if constexpr (STEP) s_flag[i] = alv[u] != 0 ? 2 : 0;
+        bad |= seqv[u] != sid[i] / a.hkv;
+      }
+    }
+    for (int i = b0 + kFirst; i < e0; ++i) {
       const int seq = a.seq_ids[i / a.hkv];
       if constexpr (STEP) {
         const int al = alpha_at(a.step.asrc, (size_t)(i / a.hkv), i % a.hkv);
@@ -1106,8 +1287,12 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     // Both control words are kept in registers until the loop's loads are out:
     // a shared-memory store of a loaded value here would hold them back one
     // round trip.
-    const int status = tid == 0 ? read_status(a.ctrl) : 0;
-    const int free_depth = (STEP && tid == 0) ? *reinterpret_cast<const volatile int32_t*>(&a.ctrl[kCtrlFree]) : 0;
+    const int status = tid == 0 ? launch_status() : 0;
+    const int free_depth = (STEP && tid == 0) ? read_word(&a.ctrl[kCtrlFree + a.par]) : 0;
+    // The current counts: the parity the host passed, else (a launch captured
+    // into a graph) the cache's parity word, read in this round trip.
+    if (cpar < 0) cpar = read_par(a.ctrl);
+    const int32_t* ncur = a.n + (size_t)cpar * a.n_stride;
     bool miss = !STEP || trust == 0;
     int local = 0;
     for (int i = b0; i < e0; ++i) {
@@ -1116,8 +1301,8 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       int4 en = make_int4(0, 0, 0, -1);
       unsigned long long etag = 0;
       if (STEP && trust != 0) {
-        en = ld_early4(reinterpret_cast<const int4*>(a.step.next.entry + i));
-        etag = ld_early_u64(&a.step.next.entry[i].tag);
+        en = ld_early4(reinterpret_cast<const int4*>(tentries + i));
+        etag = ld_early_u64(&tentries[i].tag);
       }
       int pages = 0, st = 0;
       if (seq < 0 || seq >= a.max_seqs) {
@@ -1131,10 +1316,10 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       } else {
         st = seq * a.hkv + i % a.hkv;
         const bool hit = STEP && trust != 0 && etag == trust && en.w == seq;
-        const int nn = hit ? en.x : a.n[st];
+        const int nn = clamp_count(hit ? en.x : ncur[st], a.mps, a.ctrl);
         pages = (nn + kPage - 1) / kPage;
         if constexpr (STEP) {
-          const int ps = hit ? en.y : a.step.dv.pos[st];
+          const int ps = hit ? en.y : a.step.dv.pos[(size_t)cpar * a.step.dv.S + st];
           s_nold[i] = nn;
           s_pos[i] = ps;
           s_flag[i] = al != 0 ? 2 : 0;
@@ -1157,6 +1342,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     if (tid == 0) {
       prefix[0] = 0;
       misc[1] = (status == 0);
+      misc[16] = status;
       if (STEP) misc[12] = free_depth;
     }
     any_miss = __syncthreads_or(miss) != 0;
@@ -1192,7 +1378,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   uint64_t* myfull = full + (warp < NCW ? warp : 0) * spw;
 
   if (STEP && warp == NCW) {
-    step_warp<D, E>(a, nst, prefix, sid, s_nold, s_pos, s_rslot, s_tslot, s_flag, s_rank, misc, healthy,
+    step_warp<D, E>(a, nst, prefix, sid, s_nold, s_pos, s_rslot, s_tslot, s_flag, s_rank, misc, bits, healthy,
                     abort_flag, K0, K1);
   } else if (STEP || has_range) {
     // ---- this warp's page pipeline: CTA pages c = warp + NCW * j, j = 0 .. njobs-1
@@ -1212,6 +1398,8 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       if (STEP && list_ok) return checked(__ldg(tlist + warp + NCW * j));
       const int kk = K0 + warp + NCW * j;
       const int i = stream_of(prefix, nst, kk);
+      if (!in_bounds(sid[i], (long long)a.max_seqs * a.hkv, a.ctrl) || !in_bounds(kk - prefix[i], a.mps, a.ctrl))
+        return 0;
       return checked(__ldg(a.page_table + (size_t)sid[i] * a.mps + (kk - prefix[i])));
     };
     using State = typename std::conditional<MMA, MmaState<D>, SimtState<D>>::type;
@@ -1239,7 +1427,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       for (int q = 0; q < kRingPer; ++q) {
         const int il = tid + q * kMergeThreads;
         ring_v[q] = (il < nst && s_rslot[il] == kRslotUnknown)
-                        ? ld_early(a.step.dv.ring + (size_t)sid[il] * a.step.dv.w + (s_pos[il] % a.step.dv.w))
+                        ? ld_early(a.step.dv.ring + ring_leaving(a.step.dv, sid[il], s_pos[il]))
                         : 0;
       }
     }
@@ -1280,9 +1468,10 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     if (has_range) {
 
 
+      const int32_t* ncur = a.n + (size_t)cpar * a.n_stride;
       auto retained_of = [&](int stream) -> int {   // retained count the attention runs over
         if constexpr (STEP) return s_nold[stream];
-        else return __ldg(a.n + sid[stream]);
+        else return clamp_count(__ldg(ncur + sid[stream]), a.mps, a.ctrl);
       };
       const MmaOffsets<D> off(lane);
       int k = K0;
@@ -1302,6 +1491,9 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
         const int pe = min(pend, K1);
         const int b = i / a.hkv, kvh = i % a.hkv;
         const bool whole = (k == pstart) && (pe == pend);
+        // STEP: tell the step warp the range's last piece has begun (it then reads
+        // whether the stream's other pieces are all published).
+        if (STEP && pe == K1 && tid == 0) *reinterpret_cast<volatile int*>(&misc[17]) = 1;
         const int rslot = STEP ? s_rslot[i] : -1;   // row of the token leaving at this step
         auto rows_of = [&](int p) -> uint32_t {      // rows to attend in page p of the stream
           const int valid = (pstart + p == pend - 1) ? nn - kPage * p : kPage;
@@ -1370,7 +1562,8 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
         const bool add_new = STEP && may_finish && s_tslot[i] >= 0;   // the stream's new token (appended by this step)
         float4 myO[kIters];
         float myM[kIters], myL[kIters];
-        Partial<D>* part = reinterpret_cast<Partial<D>*>(a.part) + (blockIdx.x + i);
+        Partial<D>* part = reinterpret_cast<Partial<D>*>(a.part) +
+                           (in_bounds(blockIdx.x + i, a.part_slots, a.ctrl) ? blockIdx.x + i : 0);
 #pragma unroll
         for (int it = 0; it < kIters; ++it) {
           const int t = tid + it * kMergeThreads;
@@ -1431,6 +1624,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
             if (shortcut || misc[2]) {
               const Partial<D>* base = reinterpret_cast<const Partial<D>*>(a.part) + i;
               const int me = blockIdx.x;
+              const int last_ok = in_bounds((long long)last + i, a.part_slots, a.ctrl) ? last : first - 1;
 #pragma unroll
               for (int it = 0; it < kIters; ++it) {
                 const int t = tid + it * kMergeThreads;
@@ -1441,13 +1635,13 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
                 if constexpr (STEP && MMA) fetch_new_token<D, E>(a, i, h, d4, nt);
                 float M = live ? myM[it] : 0.f, L = live ? myL[it] : 1.f;
                 float4 O = live ? myO[it] : make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int c0 = first; c0 <= last; c0 += 4) {   // loads of 4 pieces in flight at once
+                for (int c0 = first; c0 <= last_ok; c0 += 4) {   // loads of 4 pieces in flight at once
                   float mc[4], lc[4];
                   float4 oc[4];
 #pragma unroll
                   for (int u = 0; u < 4; ++u) {
                     const int c = c0 + u;
-                    const bool use = c <= last && c != me;
+                    const bool use = c <= last_ok && c != me;
                     mc[u] = use ? __ldcg(&base[c].m[h]) : -INFINITY;
                     lc[u] = use ? __ldcg(&base[c].l[h]) : 0.f;
                     oc[u] = use ? __ldcg(reinterpret_cast<const float4*>(&base[c].O[h][4 * d4]))
@@ -1507,9 +1701,17 @@ KernelFn pick_kernel(int d, int dtype, int kernel, int ncw, int nb) {
   return pick_ncw<1, false, float, STEP>(d, ncw);
 }
 
+// Launch-shape overrides for tuning sweeps. Only a build with DMS_TUNING defined
+// reads them; the library as shipped always takes the defaults, which are the
+// shapes its tests cover.
 int env_int(const char* name, int dflt) {
+#ifdef DMS_TUNING
   const char* v = getenv(name);
   return (v && *v) ? atoi(v) : dflt;
+#else
+  (void)name;
+  return dflt;
+#endif
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1547,7 +1749,16 @@ cudaError_t prepare(const Dev& dv, int dtype, int kernel_choice, int num_sms, bo
   plan->fn = reinterpret_cast<void*>(fn);
   plan->threads = (ncw + (step ? 1 : 0)) * 32;
   plan->smem = (size_t)smem_layout(ncw, spw, stage_bytes, dv.d, dv.S, step).total;
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan->smem);
+  // The dynamic shared-memory limit is an attribute of the kernel function,
+  // shared by every plan (every cache, every allocation-free call) that uses this
+  // instantiation. It is set to the device's opt-in maximum, which every plan
+  // fits under, so no plan's set-up can shrink the limit under another's launch.
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, fn);
+  if (e != cudaSuccess) return e;
+  const int limit = per_block_smem - (int)fa.sharedSizeBytes;
+  if ((int)plan->smem > limit) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
@@ -1591,18 +1802,21 @@ cudaError_t step_prepare(const Dev& dv, int dtype, int kernel_choice, int num_sm
 namespace {
 
 AttnArgs attn_args(const Dev& dv, const AttnPlan& plan, int n_seqs, const int32_t* seq_ids, const void* Q,
-                   int hq, float scale, void* out, int out_f32) {
+                   int hq, float scale, void* out, int out_f32, const AttnCounts& counts) {
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   a.seq_ids = seq_ids;
   a.Q = (const uint8_t*)Q;
   a.out = (uint8_t*)out;
-  a.n = dv.n;
+  a.n = counts.n;
+  a.n_stride = counts.stride;
+  a.par = counts.par;
   a.page_table = dv.page_table;
   a.kv = dv.kv;
   a.ctrl = dv.ctrl;
   a.part = dv.part;
   a.cnt = dv.cnt;
+  a.part_slots = dv.part_slots;
   a.n_seqs = n_seqs;
   a.hkv = dv.hkv;
   a.g = hq / dv.hkv;
@@ -1621,30 +1835,34 @@ AttnArgs attn_args(const Dev& dv, const AttnPlan& plan, int n_seqs, const int32_
 
 cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,
                              const int32_t* seq_ids, const void* Q, int hq, float scale, void* out,
-                             int out_f32, const AttnGuess& guess) {
+                             int out_f32, const AttnCounts& counts, const AttnGuess& guess) {
   if (n_seqs == 0) return cudaSuccess;
-  AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32);
+  AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32, counts);
   a.guess_rd = guess.rd;
   a.guess_wr = guess.wr;
-  a.pre_attn = guess.early && guess.rd && guess.wr ? 1 : 0;
+  // The early plan reads the counts before the dependency wait: only with the parity known.
+  a.pre_attn = guess.early && guess.rd && guess.wr && counts.par >= 0 ? 1 : 0;
   return launch_dependent(reinterpret_cast<KernelFn>(plan.fn), dim3(plan.grid), dim3(plan.threads), plan.smem, st,
                           a, plan.tmap);
 }
 
 cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
-                        const void* K, const void* V, const uint8_t* alpha, int alpha_channel, const void* Q, int hq,
-                        float scale, void* out, int out_f32, unsigned long long launch_index,
-                        const NextPlan& next, unsigned long long trust_tag, unsigned long long write_tag,
-                        bool early) {
-  if (n_seqs == 0) return cudaSuccess;
+                        const void* K, const void* V, const AlphaChoice& alpha, const void* Q, int hq,
+                        float scale, void* out, int out_f32, int par, const NextPlan& next,
+                        unsigned long long trust_tag, unsigned long long write_tag, bool early) {
+  // Every launch flips the cache's state parity, so an empty call must not get here
+  // (the host would count a flip that never happens).
+  if (n_seqs <= 0) return cudaErrorInvalidValue;
   // A schedule is read from the buffer of its tag's parity and written to the
   // other one, so the two tags must be consecutive.
   if (write_tag == 0 || (trust_tag != 0 && trust_tag + 1 != write_tag)) return cudaErrorInvalidValue;
-  AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32);
+  if (par != 0 && par != 1) return cudaErrorInvalidValue;
+  AttnArgs a = attn_args(dv, plan, n_seqs, seq_ids, Q, hq, scale, out, out_f32, AttnCounts{dv.n, dv.S, par});
   a.step.K = (const uint8_t*)K;
   a.step.V = (const uint8_t*)V;
-  a.step.asrc = AlphaSrc{alpha, (const uint8_t*)K, alpha_channel, dv.hkv, dv.d, dv.elem_bytes};
-  a.step.launch_index = launch_index;
+  if (alpha.channel < 0) a.step.asrc = alpha_given(alpha.alpha, dv.hkv);
+  else if (alpha.q_head < 0) a.step.asrc = alpha_from_keys(K, dv.hkv, dv.d, alpha.channel, dv.elem_bytes);
+  else a.step.asrc = alpha_from_queries(Q, dv.hkv, hq / dv.hkv, dv.d, alpha.q_head, alpha.channel, dv.elem_bytes);
   a.step.dv = dv;
   a.step.next = next;
   a.step.trust = next.entry ? trust_tag : 0ull;

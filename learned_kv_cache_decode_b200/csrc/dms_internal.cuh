@@ -18,55 +18,142 @@ constexpr int kMaxKvHeads = 256;
 
 // Where the eviction decisions of appended tokens come from: an explicit
 // uint8 array [rows][hkv] (channel < 0), or the sign of one designated
-// channel of each token's key row: alpha = 1 iff K[row][kvh][channel] > 0
-// (the eviction logit read from a repurposed key neuron; zero and NaN keep
-// the token).
+// channel of a projection row of each token (the eviction logit read from a
+// repurposed neuron; zero and NaN keep the token): alpha = 1 iff
+// X[(row * hkv + kvh) * stride + offset] > 0. For the key projection X = K
+// [rows][hkv][d], stride = d and offset = channel; for the query projection
+// X = Q [rows][hkv * g][d], stride = g * d and offset = head * d + channel,
+// `head` being the designated query head within the KV head's group.
 struct AlphaSrc {
   const uint8_t* alpha;   // [rows][hkv] when channel < 0
-  const uint8_t* K;       // [rows][hkv][d] elements
-  int channel, hkv, d, elem_bytes;
+  const uint8_t* X;       // projection rows holding the logit
+  int channel;            // < 0: explicit alpha array
+  int hkv;
+  int stride, offset;     // elements
+  int elem_bytes;
 };
 
+// alpha from an explicit uint8 array [rows][hkv].
+inline AlphaSrc alpha_given(const uint8_t* alpha, int hkv) {
+  return AlphaSrc{alpha, nullptr, -1, hkv, 0, 0, 2};
+}
+// alpha = 1 iff K[row][kvh][channel] > 0.
+inline AlphaSrc alpha_from_keys(const void* K, int hkv, int d, int channel, int elem_bytes) {
+  return AlphaSrc{nullptr, (const uint8_t*)K, channel, hkv, d, channel, elem_bytes};
+}
+// alpha = 1 iff Q[row][kvh * g + head][channel] > 0.
+inline AlphaSrc alpha_from_queries(const void* Q, int hkv, int g, int d, int head, int channel, int elem_bytes) {
+  return AlphaSrc{nullptr, (const uint8_t*)Q, channel, hkv, g * d, head * d + channel, elem_bytes};
+}
+
+// logit > 0 decided on the stored bits, so that no flush-to-zero mode can turn a
+// positive subnormal into a kept token: the sign bit is clear, the value is not
+// +0, and it is at most +inf (larger patterns are NaN).
 __device__ __forceinline__ int alpha_at(const AlphaSrc& s, size_t row, int kvh) {
   if (s.channel < 0) return s.alpha[row * s.hkv + kvh] != 0;
-  const size_t e = (row * s.hkv + kvh) * (size_t)s.d + s.channel;
-  const float logit = s.elem_bytes == 2
-                          ? __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(s.K)[e] << 16)
-                          : reinterpret_cast<const float*>(s.K)[e];
-  return logit > 0.f;
+  const size_t e = (row * s.hkv + kvh) * (size_t)s.stride + s.offset;
+  if (s.elem_bytes == 2) {
+    const uint32_t u = reinterpret_cast<const uint16_t*>(s.X)[e];
+    return u != 0u && u <= 0x7f80u;
+  }
+  const uint32_t u = reinterpret_cast<const uint32_t*>(s.X)[e];
+  return u != 0u && u <= 0x7f800000u;
 }
 
 // Control words (device int32).
+//
+// The per-stream counts n and pos and the free-stack depth exist twice, and
+// the state parity says which copy is current. Every kernel except the fused
+// decode step reads and writes the current copy in place. A fused step of
+// parity p reads copy p and writes copy 1 - p (every stream: the ones it
+// appends to, and a copy of the others), then sets the parity to 1 - p. So no
+// CTA of a fused step ever writes a word another CTA of the same launch reads,
+// and the step needs no grid-wide wait: its CTAs never wait on one another and
+// need not be resident at the same time.
+// Errors are latched likewise: the fused step of parity p reads the status
+// words kCtrlStatus and kCtrlStepErr + p and latches what its plan finds
+// (bad seq id, stream full, pool exhausted) into kCtrlStepErr + 1 - p, which
+// no CTA of the launch reads. Every other kernel reads all three words.
 enum : int {
-  kCtrlStatus = 0,   // latched dms_status, 0 = healthy
-  kCtrlFree = 1,     // free-stack depth
-  kCtrlPlanned = 2,  // words 2-3: uint64 count of fused-step CTAs done reading the pre-step
-                     // state, cumulative over the cache's fused steps (grid per launch)
+  kCtrlStatus = 0,    // latched dms_status, 0 = healthy
+  kCtrlFree = 1,      // words 1-2: free-stack depth of each parity
+  kCtrlPar = 3,       // state parity (0 or 1)
+  kCtrlStepErr = 4,   // words 4-5: errors latched by fused steps, by parity
   kCtrlWords = 8
 };
 
 // Everything a kernel needs to know about one cache (device pointers and sizes).
 struct Dev {
-  int32_t* pos;         // [S] tokens seen
-  int32_t* n;           // [S] retained tokens = logical slots in use
+  int32_t* pos;         // [2][S] tokens seen, one copy per state parity
+  int32_t* n;           // [2][S] retained tokens = logical slots in use, per parity
   int32_t* n_pages;     // [S]
   int32_t* page_table;  // [S][mps]
-  int32_t* ring;        // [S][w] (logical slot << 1) | alpha of the latest token per residue mod w
+  int32_t* ring;        // [S][w + 1] (logical slot << 1) | alpha of token t at t mod (w + 1)
   int32_t* slot_pos;    // [max_pages * 16] position held by each physical slot
-  int32_t* free_list;   // [max_pages] stack, top at ctrl[kCtrlFree] - 1
+  int32_t* free_list;   // [max_pages] stack, top at the current free-stack depth - 1
   int32_t* ctrl;        // [kCtrlWords]
   int32_t* scratch;     // [S] per-call scratch (append bookkeeping)
   uint8_t* kv;          // [max_pages][2][16][d] elements: 16 K rows then 16 V rows per page
   float* part;          // split-K partials [(grid + S)][8][d + 2]
   int32_t* cnt;         // [S] split-K arrival counters
   int S, hkv, d, w, mps, max_pages, max_seqs, elem_bytes;
+  int part_slots;       // partial slots in `part`
 };
+
+// Window-ring index of token t: the ring keeps w + 1 entries, so that the entry
+// of the token that may leave at step s (s - w) and the entry the new token s
+// writes are never the same word.
+// (Unsigned arithmetic: no position can give a negative index.)
+__device__ __forceinline__ size_t ring_at(const Dev& dv, int stream, int t) {
+  return (size_t)stream * (dv.w + 1) + (size_t)((uint32_t)t % (uint32_t)(dv.w + 1));
+}
+// Entry of the token that leaves when token s arrives, s - w, for s >= w.
+__device__ __forceinline__ size_t ring_leaving(const Dev& dv, int stream, int s) {
+  return (size_t)stream * (dv.w + 1) + (size_t)(((uint32_t)s + 1u) % (uint32_t)(dv.w + 1));
+}
 
 __device__ __forceinline__ void latch(int32_t* ctrl, int code) {
   atomicCAS(&ctrl[kCtrlStatus], 0, code);
 }
+
+// Bounds checks of the debug build. A library built with DMS_DEBUG defined
+// checks every index the kernels derive by construction (page-table rows and
+// columns, partial slots, pool rows, free-stack positions) against its buffer:
+// an index out of range latches DMS_ERR_INVALID and the access is skipped,
+// never a trap. In the normal build the check compiles to `true`.
+#ifdef DMS_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool in_bounds(long long idx, long long limit, int32_t* ctrl) {
+  if constexpr (kDebugChecks) {
+    if (idx < 0 || idx >= limit) {
+      latch(ctrl, DMS_ERR_INVALID);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void latch_word(int32_t* word, int code) { atomicCAS(word, 0, code); }
+__device__ __forceinline__ int read_word(const int32_t* p) { return *reinterpret_cast<const volatile int32_t*>(p); }
+// Status as every kernel but the fused step sees it: the first error latched anywhere.
 __device__ __forceinline__ int read_status(const int32_t* ctrl) {
-  return *reinterpret_cast<const volatile int32_t*>(&ctrl[kCtrlStatus]);
+  const int s = read_word(&ctrl[kCtrlStatus]);
+  const int e0 = read_word(&ctrl[kCtrlStepErr]);
+  const int e1 = read_word(&ctrl[kCtrlStepErr + 1]);
+  return s != 0 ? s : (e0 != 0 ? e0 : e1);
+}
+__device__ __forceinline__ int read_par(const int32_t* ctrl) { return read_word(&ctrl[kCtrlPar]) & 1; }
+
+// The current copies of the per-stream counts and the free-stack depth.
+struct Cur {
+  int32_t* n;
+  int32_t* pos;
+  int32_t* free;
+};
+__device__ __forceinline__ Cur cur_state(const Dev& dv, int par) {
+  return Cur{dv.n + (size_t)par * dv.S, dv.pos + (size_t)par * dv.S, dv.ctrl + kCtrlFree + par};
 }
 
 // ---------------------------------------------------------------------------
@@ -334,28 +421,6 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
-// 64-bit device-scope add with release semantics, no return value.
-__device__ __forceinline__ void red_add_release_gpu_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-// Spin (one thread) until *counter >= target, sleeping between polls, bounded
-// like wait_flag_ge.
-__device__ __forceinline__ void wait_count_ge(const volatile unsigned long long* counter, unsigned long long target,
-                                              volatile int* abort_flag, int32_t* ctrl, int sleep_ns) {
-  if (*counter >= target) return;
-  const long long t0 = clock64();
-  while (*counter < target) {
-    __nanosleep(sleep_ns);
-    if (*abort_flag) return;
-    if (clock64() - t0 > (1ll << 31)) {
-      latch(ctrl, DMS_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return;
-    }
-  }
-}
-
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -366,17 +431,17 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
 cudaError_t prepare_aux_kernels();
 cudaError_t launch_init_state(const Dev& dv, cudaStream_t st);
 cudaError_t launch_append_decode(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
-                                 const void* K, const void* V, const uint8_t* alpha, int alpha_channel,
-                                 int* launches);
+                                 const void* K, const void* V, const AlphaSrc& asrc, int* launches);
 cudaError_t launch_append_bulk(const Dev& dv, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
                                const int32_t* cu_tokens, int total_tokens, const void* K, const void* V,
-                               const uint8_t* alpha, int alpha_channel, int* launches);
+                               const AlphaSrc& asrc, int* launches);
 cudaError_t launch_reset_seq(const Dev& dv, cudaStream_t st, int seq);
 cudaError_t launch_bounded_wait_selftest(const Dev& dv, cudaStream_t st, int32_t* timed_out);
 cudaError_t launch_stats(const Dev& dv, cudaStream_t st, int32_t* retained, int32_t* seen, float* head_cr,
                          int64_t* totals);
 cudaError_t launch_gather(const Dev& dv, cudaStream_t st, int seq, int kvh, int rows_cap, void* Kout,
                           void* Vout);
+cudaError_t launch_alpha_from_logit(cudaStream_t st, const AlphaSrc& src, int rows, uint8_t* out);
 
 // Decode attention plan shared by host and launcher.
 struct AttnPlan {
@@ -416,22 +481,31 @@ struct __align__(16) PlanEntry {
 // Page list of CTA c for the next step: the physical page ids of its range, in
 // range order, with a header of two int4: {tag lo, tag hi, call streams, total
 // pages} and {range begin, range end, 0, 0}.
-// Double-buffered by tag parity: a step reads the buffer of the tag it trusts
-// while it writes the other one.
+// Entries and lists are double-buffered by tag parity: a step reads the buffers
+// of the tag it trusts while it writes the other ones.
 struct NextPlan {
-  PlanEntry* entry;   // [S]
+  PlanEntry* entry;   // [2][S]
   int4* hdr;          // [2][grid][2]
   int32_t* list;      // [2][grid][cap]
   int cap;            // page ids per CTA: enough for any range of any call (max_pages / grid, rounded up)
+  int S;              // entries per tag parity
 };
-// `early`: the host knows that the kernel just before this launch in its stream
-// does not write this cache, so the step may plan from the schedule and start
-// its first page copies before its dependency wait (checked after it).
+// Where the eviction decisions of a fused step's new tokens come from: an
+// alpha array (channel < 0), or the sign of channel `channel` of the key row
+// (q_head < 0) or of query head `q_head` of the KV head's group.
+struct AlphaChoice {
+  const uint8_t* alpha;
+  int channel;
+  int q_head;
+};
+// `par`: the cache's state parity before this step (the host counts the fused
+// steps). `early`: the host knows that the kernel just before this launch in
+// its stream does not write this cache, so the step may plan from the schedule
+// and start its first page copies before its dependency wait (checked after it).
 cudaError_t launch_step(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs, const int32_t* seq_ids,
-                        const void* K, const void* V, const uint8_t* alpha, int alpha_channel, const void* Q, int hq,
-                        float scale, void* out, int out_f32, unsigned long long launch_index,
-                        const NextPlan& next, unsigned long long trust_tag, unsigned long long write_tag,
-                        bool early);
+                        const void* K, const void* V, const AlphaChoice& alpha, const void* Q, int hq,
+                        float scale, void* out, int out_f32, int par, const NextPlan& next,
+                        unsigned long long trust_tag, unsigned long long write_tag, bool early);
 constexpr int kStepMaxStreams = 1024;   // caches with more streams run the step as two launches
 
 // The stream list of the previous attention call on a cache, kept on the device
@@ -445,8 +519,17 @@ struct AttnGuess {
   int32_t* wr;         // this call's list, for the next call
   bool early;
 };
+// Retained counts the attention reads: `n` + parity * `stride`, the parity being
+// `par` when it is >= 0, else read from the cache's parity word (a launch into a
+// stream under capture runs later, after fused steps the host cannot foresee).
+// Caller-owned counts: stride 0, par 0.
+struct AttnCounts {
+  const int32_t* n;
+  int stride;
+  int par;
+};
 cudaError_t launch_attention(const Dev& dv, const AttnPlan& plan, cudaStream_t st, int n_seqs,
                              const int32_t* seq_ids, const void* Q, int hq, float scale, void* out,
-                             int out_f32, const AttnGuess& guess);
+                             int out_f32, const AttnCounts& counts, const AttnGuess& guess);
 
 }  // namespace dms

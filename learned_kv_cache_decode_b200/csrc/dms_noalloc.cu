@@ -32,17 +32,27 @@ static_assert(kPartOffset % 256 == 0, "partials must start 256-aligned");
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
+constexpr int kPlans = 8;   // launch plans kept per device
 
-// Per-device set-up, done by the first call on that device.
+// A launch plan and what it was made for (the tensor map holds the pool's
+// address and size; the shared-memory plan arrays are sized by the streams).
+struct CachedPlan {
+  bool valid = false;
+  unsigned long long used = 0;   // last use, for replacement
+  AttnPlan plan;
+  const void* pool = nullptr;
+  int d = 0, dtype = 0, streams = 0, max_pages = 0;
+};
+
+// Per-device set-up, done by the first call on that device, and the plans of
+// the last few distinct call shapes, so that a caller alternating between
+// batch sizes or pools does not prepare a plan on every call.
 struct DeviceState {
   bool ready = false;
   unsigned char* scratch = nullptr;   // device address of g_scratch
   int num_sms = 0;
-  // plan of the last call, reused while its inputs are the same
-  bool have_plan = false;
-  AttnPlan plan;
-  const void* pool = nullptr;
-  int d = 0, dtype = 0, streams = 0, max_pages = 0;
+  unsigned long long clock = 0;
+  CachedPlan plans[kPlans];
 };
 
 std::mutex g_mu;
@@ -99,21 +109,30 @@ static dms_status noalloc_impl(cudaStream_t stream, const dms_paged_kv* kv, int3
       if (cudaDeviceGetAttribute(&ds.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DMS_ERR_CUDA;
       ds.ready = true;
     }
-    if (!ds.have_plan || ds.pool != kv->kv_pool || ds.d != d || ds.dtype != (int)kv->dtype ||
-        ds.streams != (int)nst || ds.max_pages != kv->max_pages) {
-      cudaError_t e = attention_prepare(dv, kv->dtype, DMS_ATTN_AUTO, ds.num_sms, &ds.plan);
-      if (e != cudaSuccess) {
-        ds.have_plan = false;
-        return e == cudaErrorInvalidValue ? DMS_ERR_INVALID : DMS_ERR_CUDA;
+    CachedPlan* hit = nullptr;
+    CachedPlan* victim = &ds.plans[0];
+    for (CachedPlan& c : ds.plans) {
+      if (c.valid && c.pool == kv->kv_pool && c.d == d && c.dtype == (int)kv->dtype && c.streams == (int)nst &&
+          c.max_pages == kv->max_pages) {
+        hit = &c;
+        break;
       }
-      ds.have_plan = true;
-      ds.pool = kv->kv_pool;
-      ds.d = d;
-      ds.dtype = (int)kv->dtype;
-      ds.streams = (int)nst;
-      ds.max_pages = kv->max_pages;
+      if (!c.valid || (victim->valid && c.used < victim->used)) victim = &c;
     }
-    plan = ds.plan;
+    if (hit == nullptr) {
+      victim->valid = false;
+      cudaError_t e = attention_prepare(dv, kv->dtype, DMS_ATTN_AUTO, ds.num_sms, &victim->plan);
+      if (e != cudaSuccess) return e == cudaErrorInvalidValue ? DMS_ERR_INVALID : DMS_ERR_CUDA;
+      victim->valid = true;
+      victim->pool = kv->kv_pool;
+      victim->d = d;
+      victim->dtype = (int)kv->dtype;
+      victim->streams = (int)nst;
+      victim->max_pages = kv->max_pages;
+      hit = victim;
+    }
+    hit->used = ++ds.clock;
+    plan = hit->plan;
     scratch = ds.scratch;
   }
   // Every piece of a split stream needs a partial slot: (CTA, stream) pairs
@@ -123,12 +142,14 @@ static dms_status noalloc_impl(cudaStream_t stream, const dms_paged_kv* kv, int3
   dv.ctrl = reinterpret_cast<int32_t*>(scratch);
   dv.cnt = reinterpret_cast<int32_t*>(scratch + kCtrlBytes);
   dv.part = reinterpret_cast<float*>(scratch + kPartOffset);
+  dv.part_slots = DMS_NOALLOC_MAX_PIECES;
   // The status word and the arrival counters must start at zero; a previous
   // call leaves the counters at zero, but one that stopped on a device-side
   // error may not. The partials are written before they are read.
   if (cudaMemsetAsync(scratch, 0, kCtrlBytes + (size_t)nst * 4, stream) != cudaSuccess) return DMS_ERR_CUDA;
   cudaError_t e = launch_attention(dv, plan, stream, n_seqs, seq_ids, Q, num_q_heads, scale, out,
-                                   out_dtype == DMS_F32, AttnGuess{nullptr, nullptr, false});
+                                   out_dtype == DMS_F32, AttnCounts{kv->retained, 0, 0},
+                                   AttnGuess{nullptr, nullptr, false});
   return e == cudaSuccess ? DMS_OK : DMS_ERR_CUDA;
 }
 

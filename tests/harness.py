@@ -12,7 +12,7 @@ import numpy as np
 import torch
 
 import oracle
-from learned_kv_cache_decode_b200 import DmsCache
+from learned_kv_cache_decode_b200 import DmsCache, alpha_from_logit
 from learned_kv_cache_decode_b200 import workloads as W
 
 MAX_ABS = 2e-2     # tolerance on bf16 inputs, max |gpu - oracle|
@@ -39,12 +39,19 @@ class Run:
     """One workload on one cache plus its oracle simulator, call for call."""
 
     def __init__(self, wl: W.Workload, attn_kernel: str = "auto", steps: int | None = None,
-                 max_pages: int | None = None, check_sim: bool = True, alpha_channel: int | None = None):
+                 max_pages: int | None = None, check_sim: bool = True, alpha_channel: int | None = None,
+                 alpha_query: tuple[int, int] | None = None):
         """alpha_channel: the library reads every token's alpha from the sign of this key
         channel (dms_append_keyed / dms_decode_step_keyed); the oracle gets the same bits
-        from oracle.alpha_from_keys."""
+        from oracle.alpha_from_keys.
+        alpha_query = (head, channel): the decode tokens' alpha comes from that channel of
+        that query head of each group in the step's queries (dms_decode_step_qkeyed, or
+        dms_alpha_from_logit then dms_append); the oracle gets the same bits from
+        oracle.alpha_from_queries. The prompt's alpha is the workload's."""
         self.wl = wl
         self.alpha_channel = alpha_channel
+        self.alpha_query = alpha_query
+        self.dec_alpha = {}   # (seq, position) -> alpha row of a decode token taken from the queries
         self.ctx = W.contexts(wl)
         self.steps = wl.decode_steps if steps is None else steps
         mp, mps = pool_pages(wl, self.ctx, self.steps)
@@ -115,6 +122,10 @@ class Run:
         V = np.stack([t[1] for t in toks])
         A = np.stack([t[2] for t in toks])
         Q = W.query(self.wl, step)[list(seqs)]
+        if self.alpha_query is not None:
+            A = oracle.alpha_from_queries(Q, self.wl.num_kv_heads, *self.alpha_query)
+            for j, b in enumerate(seqs):
+                self.dec_alpha[(b, int(self.seen[b]))] = A[j]
         return K, V, A, Q
 
     def decode_step(self, step: int, seqs=None, out_dtype=None, fused: bool = False):
@@ -124,6 +135,24 @@ class Run:
         K, V, A, Q = self.decode_inputs(step, seqs)
         ids = torch.tensor(seqs, dtype=torch.int32, device="cuda")
         dev_alpha = None if self.alpha_channel is not None else torch.from_numpy(A).cuda()
+        if self.alpha_query is not None:
+            head, channel = self.alpha_query
+            dQ = to_device(Q, self.wl)
+            if fused:
+                out = self.cache.decode_step(ids, to_device(K, self.wl), to_device(V, self.wl), None, dQ,
+                                             scale=self.scale, out_dtype=out_dtype, alpha_channel=channel,
+                                             alpha_head=head)
+            else:
+                a_dev = alpha_from_logit(dQ, self.wl.num_kv_heads, channel, head)
+                np.testing.assert_array_equal(a_dev.cpu().numpy(), A)   # the decisions, bit for bit
+                self.cache.append(ids, to_device(K, self.wl), to_device(V, self.wl), a_dev)
+                out = self.cache.decode_attention(ids, dQ, scale=self.scale, out_dtype=out_dtype)
+            if self.sim is not None:
+                rc, _ = self.sim.append(seqs, [1] * len(seqs), A)
+                assert rc == 0, rc
+            for b in seqs:
+                self.seen[b] += 1
+            return out, Q
         if fused:
             out = self.cache.decode_step(ids, to_device(K, self.wl), to_device(V, self.wl), dev_alpha,
                                          to_device(Q, self.wl), scale=self.scale, out_dtype=out_dtype,
@@ -150,7 +179,39 @@ class Run:
         T = int(self.seen[b])
         K, V = W.kv(self.wl, b, 0, T)
         A = self.alpha_of(b, 0, T, K)
+        if self.dec_alpha:
+            A = A.copy()
+            for (sb, pos), row in self.dec_alpha.items():
+                if sb == b and pos < T:
+                    A[pos] = row
         return oracle.decode_gqa(W.to_f64(q), W.to_f64(K), W.to_f64(V), A, self.wl.window, self.scale)
+
+    def oracle_all(self, Q: np.ndarray, seqs=None, group: int = 2) -> np.ndarray:
+        """Oracle outputs [len(seqs), Hq, d] of many sequences at their current last
+        positions, streams run in parallel by the oracle's batch routine, `group`
+        sequences at a time (bounded host memory)."""
+        seqs = list(range(self.wl.batch)) if seqs is None else list(seqs)
+        hkv, g = self.wl.num_kv_heads, self.wl.group
+        out = np.empty((len(seqs), self.wl.num_q_heads, self.wl.head_dim))
+        for j0 in range(0, len(seqs), group):
+            items = []
+            for j in range(j0, min(j0 + group, len(seqs))):
+                b = seqs[j]
+                T = int(self.seen[b])
+                K, V = W.kv(self.wl, b, 0, T)
+                A = self.alpha_of(b, 0, T, K)
+                if self.dec_alpha:
+                    A = A.copy()
+                    for (sb, pos), row in self.dec_alpha.items():
+                        if sb == b and pos < T:
+                            A[pos] = row
+                q, K, V = W.to_f64(Q[j]), W.to_f64(K), W.to_f64(V)
+                for k in range(hkv):
+                    items.append((q[k * g:(k + 1) * g], K[:, k], V[:, k], A[:, k]))
+            res, _ = oracle.attention_batch(items, self.wl.window, self.scale)
+            for n, j in enumerate(range(j0, min(j0 + group, len(seqs)))):
+                out[j] = np.concatenate(res[n * hkv:(n + 1) * hkv])
+        return out
 
     def check_metadata(self) -> None:
         """Page tables, counters, free stack and retained sets bit-exact against the simulator."""

@@ -2,8 +2,9 @@
 
 Metadata (page tables, counters, free stack, retained sets of every
 stream) is compared bit for bit after the prefill and at checkpoints;
-attention outputs are compared on sampled (step, sequence) pairs, all query
-heads, against the fp64 oracle in definition form.
+attention outputs are compared on sampled (step, sequence) pairs and for
+every sequence at the last step, all query heads, against the fp64 oracle in
+definition form.
 """
 import numpy as np
 import pytest
@@ -17,6 +18,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _run_config(name, check_steps, check_seqs, steps=None, chunk=4096, metadata_every=None, fused=False):
+    """Sampled sequences at the steps in check_steps, and every sequence at the last step."""
     wl = W.WORKLOADS[name]
     run = Run(wl, steps=steps)
     try:
@@ -25,7 +27,12 @@ def _run_config(name, check_steps, check_seqs, steps=None, chunk=4096, metadata_
         n = run.steps
         for step in range(n):
             out, Q = run.decode_step(step, fused=fused)
-            if step in check_steps:
+            if step == n - 1:
+                torch.cuda.synchronize()
+                ref = run.oracle_all(Q)
+                for b in range(wl.batch):
+                    compare(out[b], ref[b])
+            elif step in check_steps:
                 torch.cuda.synchronize()
                 for b in check_seqs:
                     compare(out[b], run.oracle_out(b, Q[b]))

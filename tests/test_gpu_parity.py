@@ -9,6 +9,8 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
+from learned_kv_cache_decode_b200 import alpha_from_logit
 from learned_kv_cache_decode_b200 import workloads as W
 from learned_kv_cache_decode_b200 import _native
 from harness import Run, compare, to_device
@@ -94,6 +96,27 @@ def test_stats_match_oracle_counts():
         for h in range(case.num_kv_heads):
             ref = o["pos"][h::case.num_kv_heads].sum() / o["n"][h::case.num_kv_heads].sum()
             assert abs(float(st["head_cr"][h]) - ref) <= 1e-6 * ref
+    finally:
+        run.close()
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["two_launches", "fused_step"])
+def test_stats_host_matches_oracle_counts(fused):
+    """dms_stats_host: host per-stream counts and the overall CR (fp64) equal to the
+    simulator's, after decode steps of either path (a fused step flips the state parity
+    the host copies from)."""
+    case = wl("stats-host", 4, 8, 2, 64, "bf16", 16, (10, 500), 3, 0.6, 23)
+    run = Run(case)
+    try:
+        run.prefill()
+        for step in range(3):
+            run.decode_step(step, fused=fused)
+            st = run.cache.stats_host()
+            o = run.sim.snapshot()
+            np.testing.assert_array_equal(st["retained"], o["n"])
+            np.testing.assert_array_equal(st["seen"], o["pos"])
+            assert st["cr_overall"] == float(o["pos"].sum()) / float(o["n"].sum())
+        assert run.cache.status() == _native.DMS_OK
     finally:
         run.close()
 
@@ -400,7 +423,9 @@ SWEEP_WINDOWS = [1, 2, 16, 32, 64, 128, 256]
 @pytest.mark.parametrize("w", SWEEP_WINDOWS)
 @pytest.mark.parametrize("fused", [False, True], ids=["two_launches", "fused_step"])
 def test_window_sweep(w, fused):
-    """The delayed-eviction window swept from immediate eviction (w = 1, reading R15) to
+    """The delayed-eviction window swept from immediate eviction (w = 1: a marked token is
+    attended by its own step's query only, the plainest reading of the paper's
+    immediate-eviction ablation, section 5.3 and Fig. 5) to
     256, on one workload shape, through both decode paths: metadata bit for bit, every
     output against the oracle."""
     case = wl(f"sweep-w{w}", 3, 21, 3, 128, "bf16", w, (300, 900), 6, 0.7, 42)
@@ -694,3 +719,59 @@ def test_keyed_entry_points_reject_a_channel_outside_head_dim():
         assert e.value.code == _native.DMS_ERR_INVALID
     finally:
         run.close()
+
+
+# ---------------------------------------------------------------------------
+# alpha read from a designated query channel (dms_decode_step_qkeyed, dms_alpha_from_logit)
+
+QKEYED = [
+    (wl("qkeyed-bf16-g7-d128", 3, 21, 3, 128, "bf16", 16, (1, 700), 6, 0.5, 46), (6, 5)),
+    (wl("qkeyed-bf16-g4-d64-w1", 2, 8, 2, 64, "bf16", 1, (20, 300), 5, 0.5, 47), (0, 63)),
+    (wl("qkeyed-f32-g4-d64", 2, 8, 2, 64, "f32", 4, (1, 400), 6, 0.5, 48), (3, 0)),
+]
+
+
+@pytest.mark.parametrize("case,pick", QKEYED, ids=[c.name for c, _ in QKEYED])
+@pytest.mark.parametrize("fused", [False, True], ids=["two_launches", "fused_step"])
+def test_alpha_from_query_channel(case, pick, fused):
+    """Every decode token's alpha comes from channel c of query head j of its KV head's
+    group in the step's queries: fused (dms_decode_step_qkeyed) or dms_alpha_from_logit
+    (checked bit for bit against oracle.alpha_from_queries) then dms_append. Metadata bit
+    for bit, outputs within tolerance of the oracle fed the same bits."""
+    run = Run(case, alpha_query=pick)
+    tol = dict(max_abs=1e-4, mean_abs=1e-5) if case.dtype == "f32" else {}
+    try:
+        run.prefill(chunk=97)
+        for step in range(case.decode_steps):
+            out, Q = run.decode_step(step, fused=fused)
+            torch.cuda.synchronize()
+            for b in range(case.batch):
+                compare(out[b], run.oracle_out(b, Q[b]), **tol)
+            run.check_metadata()
+        marks = sum(int(a.sum()) for a in run.dec_alpha.values())
+        assert 0 < marks < len(run.dec_alpha) * case.num_kv_heads   # both decisions occur
+        assert run.cache.status() == _native.DMS_OK
+    finally:
+        run.close()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_alpha_from_logit_special_values_bit_exact(dtype):
+    """dms_alpha_from_logit on keys (one head per KV head) and on queries (a group of
+    g), on random logits mixed with +-0, subnormals, +-inf and NaN: bit for bit equal to
+    the oracle's sign rule."""
+    gen = np.random.default_rng(49)
+    rows, hkv, g, d = 257, 3, 4, 64
+    X = gen.standard_normal((rows, hkv * g, d)).astype(np.float32)
+    special = np.array([0.0, -0.0, 1e-40, -1e-40, np.inf, -np.inf, np.nan, 1.0, -1.0], dtype=np.float32)
+    X[:, :, 7] = special[gen.integers(0, len(special), size=(rows, hkv * g))]
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    Xt = torch.from_numpy(X).to(tdt)
+    Xh = Xt.numpy() if dtype == "f32" else Xt.view(torch.int16).numpy().view(np.uint16)
+    Xd = Xt.cuda()
+    for head, ch in ((0, 7), (3, 7), (2, 11)):
+        got = alpha_from_logit(Xd, hkv, ch, head).cpu().numpy()
+        np.testing.assert_array_equal(got, oracle.alpha_from_queries(Xh, hkv, head, ch))
+    K = Xd[:, :hkv].contiguous()   # keys: one head per KV head
+    got = alpha_from_logit(K, hkv, 7).cpu().numpy()
+    np.testing.assert_array_equal(got, oracle.alpha_from_keys(Xh[:, :hkv], 7))
