@@ -60,7 +60,7 @@ def test_dominant_keys_on_piece_boundaries_and_scaled_queries(dtype, kernel, d, 
     hkv, B = 2, 4
     hq = g * hkv
     T = [48, 40, 33, 80]   # tokens per sequence: several pages, ragged last pages
-    where = [[15, 16], [31, 32], [0, 39], [47, 79]]   # dominant keys: page / piece boundaries
+    where = [[15, 16], [31, 32], [0, 32], [47, 79]]   # dominant keys: page / piece boundaries
     rng = np.random.default_rng(90 + d + g + int(qs))
     scale = 1.0 / math.sqrt(d)
     Q = rng.standard_normal((B, hq, d)).astype(np.float32) * qs
