@@ -331,7 +331,7 @@ def time_oracle_one_core(items, window, scale, target_s):
 
 
 def measure(wl, args, world, rank, local, dev, *, steps, warmup, layers=0, depth=None, want_e2e=True,
-            want_cpu=False, fused=True):
+            want_cpu=False, fused=True, cpu_seconds=None):
     """Prefill L layer caches of workload `wl`, then time decode steps. Returns the
     figures of one workload (and, with want_e2e / want_cpu, its e2e and CPU passes)."""
     import torch
@@ -623,8 +623,9 @@ def measure(wl, args, world, rank, local, dev, *, steps, warmup, layers=0, depth
                                       (K_p, V_p, A_s, offs),
                                       (Kd[:, sample_seqs], Vd[:, sample_seqs], Ad_s[:, sample_seqs],
                                        Qd[:, sample_seqs]))
-        reps, t_cpu, threads = time_oracle(items, wl.window, scale, args.cpu_seconds)
-        reps1, t_cpu1 = time_oracle_one_core(items, wl.window, scale, args.cpu_seconds / 2)
+        cpu_s = args.cpu_seconds if cpu_seconds is None else cpu_seconds
+        reps, t_cpu, threads = time_oracle(items, wl.window, scale, cpu_s)
+        reps1, t_cpu1 = time_oracle_one_core(items, wl.window, scale, cpu_s / 2)
         # per decode step of the whole workload (every stream of every layer), from the sample's rate
         step_bytes = total_bytes / steps
         res["cpu"] = {
@@ -687,9 +688,13 @@ def per_workload_runs(args, world, rank, local, dev, main_wl):
         if wl.name == main_wl.name and wl == main_wl:
             continue
         t0 = time.perf_counter()
-        r = measure(wl, args, world, rank, local, dev, steps=steps, warmup=3, want_e2e=False, want_cpu=False,
-                    fused=args.step == "fused")
+        r = measure(wl, args, world, rank, local, dev, steps=steps, warmup=3, want_e2e=False,
+                    want_cpu=not args.no_cpu_baseline, fused=args.step == "fused", cpu_seconds=3.0)
         runs[name] = brief(r)
+        if "cpu" in r:   # a short oracle sample of the same step: all host cores and one core
+            runs[name]["oracle_ms_per_step"] = r["cpu"]["ms_per_step"]
+            runs[name]["oracle_ms_per_step_one_core"] = r["cpu"]["one_core"]["ms_per_step"]
+            runs[name]["oracle_cores"] = r["cpu"]["cores"]
         runs[name]["wall_s"] = time.perf_counter() - t0
     runs["tiny"] = {"note": "correctness only: one fp32 stream of about 280 retained tokens (0.15 MB per step), "
                             "checked every step against the oracle in tests/test_gpu_configs.py"}

@@ -46,14 +46,7 @@ namespace dms {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-// Stages per warp filled before the dependency wait of an early start; the
-// rest of a warp's first `spw` pages go out right after the round trip that
-// checks the guess has been issued, so that round trip is not queued behind
-// the whole first burst of page copies.
-#ifndef DMS_PRE_STAGES
-#define DMS_PRE_STAGES 8
-#endif
-constexpr int kPreStages = DMS_PRE_STAGES;
+
 constexpr int kRslotUnknown = -2;   // leaving slot not known until the window ring is read
 
 // A decode step fused into the attention launch: the new token of every call
@@ -188,18 +181,24 @@ __device__ __forceinline__ uint32_t sw128(uint32_t stage, int row, int chunk) {
 
 // Per-lane byte offsets (within a stage) of the ldmatrix rows this lane
 // addresses: K tiles for QK (rows 0..15) and V tiles for PV (rows 16..31).
+// Chunk 2t + x and chunk 2t + 8 + x lie at the same place of consecutive
+// 64-column boxes (the swizzle sees only the low three chunk bits), so the
+// offsets of the first box serve every box: offset(t) = k[t % 4] + (t / 4) * 4096.
 template <int D>
 struct MmaOffsets {
-  uint32_t k[D / 16], v[D / 16];
+  static constexpr int kN = D / 16 < 4 ? D / 16 : 4;
+  uint32_t k[kN], v[kN];
   __device__ __forceinline__ explicit MmaOffsets(int lane) {
     const int krow = lane & 15;
     const int vrow = 16 + ((lane >> 4) << 3) + (lane & 7);
 #pragma unroll
-    for (int t = 0; t < D / 16; ++t) {
+    for (int t = 0; t < kN; ++t) {
       k[t] = sw128(0, krow, 2 * t + (lane >> 4));
       v[t] = sw128(0, vrow, 2 * t + ((lane >> 3) & 1));
     }
   }
+  __device__ __forceinline__ uint32_t koff(int t) const { return k[t % kN] + (uint32_t)(t / kN) * 4096u; }
+  __device__ __forceinline__ uint32_t voff(int t) const { return v[t % kN] + (uint32_t)(t / kN) * 4096u; }
 };
 
 // NP pages of one stream at once: their QK products, one shared online-
@@ -218,7 +217,7 @@ __device__ __forceinline__ void mma_pages(MmaState<D>& S, const uint32_t (&stage
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       uint32_t af[4];
-      ldsm_x4(stage[p] + off.k[kk], af);
+      ldsm_x4(stage[p] + off.koff(kk), af);
       if (kk & 1) mma_16816(sb, af, S.qb[kk][0], S.qb[kk][1]);
       else        mma_16816(sa, af, S.qb[kk][0], S.qb[kk][1]);
     }
@@ -292,7 +291,7 @@ __device__ __forceinline__ void mma_pages(MmaState<D>& S, const uint32_t (&stage
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
       uint32_t af[4];
-      ldsm_x4_trans(stage[p] + off.v[mt], af);
+      ldsm_x4_trans(stage[p] + off.voff(mt), af);
       af[0] &= keep0;
       af[1] &= keep0;
       af[2] &= keep1;
@@ -1128,7 +1127,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     pre_k1 = k1;
     if (pre_ok && warp < NCW) {
       const int nj = k1 - k0 > warp ? (k1 - k0 - warp + NCW - 1) / NCW : 0;
-      for (int j = 0; j < spw && j < kPreStages && j < nj; ++j) {
+      for (int j = 0; j < spw && j < nj; ++j) {
         int pg = __shfl_sync(0xffffffffu, spec_pg, j);
         if (lane == 0) {
           if (pg < 0 || pg >= a.max_pages) {
@@ -1196,7 +1195,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
             pid_pre = 0;
           }
         }
-        for (int j = 0; j < spw && j < kPreStages && j < nj; ++j) {
+        for (int j = 0; j < spw && j < nj; ++j) {
           const int pg = __shfl_sync(0xffffffffu, pid_pre, j);
           if (lane == 0)
             issue_page<D, MMA, E>(full + warp * spw, smem + lay.stages + (size_t)warp * spw * kStage, spw, j, pg,
@@ -1215,40 +1214,8 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     // The call's seq ids against the guess, and (STEP) the alpha of its new
     // tokens, in the same round trip as the query of the CTA's first piece.
     if (warp < NCW && pre_k1 > pre_k0) fetch_query(stream_of(prefix, nst, pre_k0));
-    // The first streams' seq ids (and alpha) are requested before the rest of
-    // the pre-planned copies, their values used after.
-    constexpr int kFirst = 4;
-    int seqv[kFirst], alv[kFirst];
-#pragma unroll
-    for (int u = 0; u < kFirst; ++u) {
-      const int i = b0 + u;
-      seqv[u] = i < e0 ? a.seq_ids[i / a.hkv] : 0;
-      alv[u] = (STEP && i < e0) ? alpha_at(a.step.asrc, (size_t)(i / a.hkv), i % a.hkv) : 0;
-    }
-    if (kPreStages < spw && warp < NCW) {   // warp-collective (page ids shuffled from the lanes)
-      const int nj = pre_k1 - pre_k0 > warp ? (pre_k1 - pre_k0 - warp + NCW - 1) / NCW : 0;
-      for (int j = kPreStages; j < spw && j < nj; ++j) {
-        int pg = __shfl_sync(0xffffffffu, STEP ? spec_pg : pid_pre, j);
-        if (lane == 0) {
-          if (pg < 0 || pg >= a.max_pages) {
-            latch(a.ctrl, DMS_ERR_INVALID);
-            pg = 0;
-          }
-          issue_page<D, MMA, E>(full + warp * spw, smem + lay.stages + (size_t)warp * spw * kStage, spw, j, pg,
-                                &tmap, a.kv);
-        }
-      }
-    }
     bool bad = false;
-#pragma unroll
-    for (int u = 0; u < kFirst; ++u) {
-      const int i = b0 + u;
-      if (i < e0) {
-        if constexpr (STEP) s_flag[i] = alv[u] != 0 ? 2 : 0;
-        bad |= seqv[u] != sid[i] / a.hkv;
-      }
-    }
-    for (int i = b0 + kFirst; i < e0; ++i) {
+    for (int i = b0; i < e0; ++i) {
       const int seq = a.seq_ids[i / a.hkv];
       if constexpr (STEP) {
         const int al = alpha_at(a.step.asrc, (size_t)(i / a.hkv), i % a.hkv);
