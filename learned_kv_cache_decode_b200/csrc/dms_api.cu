@@ -159,9 +159,11 @@ void free_next(dms::NextPlan& np) {
 
 // Buffers of the schedules a fused step leaves for the next one: per tag
 // parity, one entry per stream and one page list per CTA of the step's grid,
-// long enough for any range (a call holds at most max_pages pages).
+// long enough for any range (a call holds at most max_pages pages in at most
+// S streams; a range spans at most 1 / grid of their weighted cost).
 cudaError_t alloc_next(const dms::Dev& dv, int grid, dms::NextPlan* np) {
-  np->cap = (int)std::max<int64_t>(1, ((int64_t)dv.max_pages + grid - 1) / grid);
+  np->cap = (int)std::max<int64_t>(
+      1, ((int64_t)dv.max_pages + (int64_t)dms::kMaxPieceCost * dv.S + grid - 1) / grid);
   np->S = dv.S;
   cudaError_t e = alloc(&np->entry, (size_t)2 * dv.S);
   if (e == cudaSuccess) e = alloc(&np->hdr, (size_t)2 * grid * 2);

@@ -110,11 +110,45 @@ __device__ __forceinline__ int stream_of(const int* prefix, int n, int x) {
   return lo;
 }
 
-// Range (CTA) that owns global page index x when P pages are cut into G
-// ranges [floor(c P / G), floor((c+1) P / G)), all of them non-empty (G <= P).
+// Part that holds point x of [0, P) when the line is cut into G parts
+// [floor(c P / G), floor((c+1) P / G)), all of them non-empty (G <= P).
 __device__ __forceinline__ int range_of(long long x, long long P, long long G) {
   return (int)(((x + 1) * G - 1) / P);
 }
+
+// The call's pages cut into CTA ranges, weighted by stream pieces. Page k of
+// call stream i sits at cost k + X i on a line of length C = P + X nst: every
+// stream adds X page-times, the merge that ends a piece of it, which a CTA
+// pays once for each stream its range touches. The line is cut into Geff =
+// min(C, G) parts [floor(b C / Geff), floor((b + 1) C / Geff)), none empty,
+// and CTA b takes the pages whose cost falls in part b: a contiguous page
+// range, empty when the part lies inside the cost of a merge, and CTAs beyond
+// Geff hold nothing. The CTAs holding pieces of one stream are consecutive.
+// With X = 0 these are the equal page ranges.
+struct Cut {
+  long long C;
+  int Geff, X;
+  __device__ __forceinline__ Cut(long long P, int nst, int x, int G) : X(x) {
+    C = P + (long long)x * nst;
+    Geff = C < G ? (int)C : G;
+  }
+  // The CTA whose range holds page k of call stream i.
+  __device__ __forceinline__ int owner(long long k, int i) const { return range_of(k + (long long)X * i, C, Geff); }
+  // First page of CTA b's range, b >= 0 (the end of range b is begin(b + 1)).
+  // pf(i): pages of the call streams before stream i, for i in [0, nst].
+  template <typename Pf>
+  __device__ __forceinline__ long long begin(int b, int nst, Pf pf) const {
+    if (b >= Geff) return pf(nst);
+    const long long T = (long long)b * C / Geff;   // < C
+    int lo = 0, hi = nst;   // the last stream whose cost starts at or before T
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pf(mid) + (long long)X * mid <= T) lo = mid; else hi = mid;
+    }
+    const long long p0 = pf(lo), into = T - (p0 + (long long)X * lo), n = pf(lo + 1) - p0;
+    return p0 + (into < n ? into : n);
+  }
+};
 
 // Partial result of one (CTA range, stream) piece: unnormalised output
 // O[head][d], running max m[head] (base-2 domain) and sum l[head]. The same
@@ -585,7 +619,7 @@ __device__ __forceinline__ void combine_stream(const AttnArgs& a, int i, int fir
 // of this launch reads (the other parity's counts, the ring entry of token s
 // rather than that of s - w, page-table entries past the pre-step pages, rows
 // the attention masks or that lie past the pre-step counts).
-template <int D, typename E>
+template <int D, typename E, int X>
 __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int* prefix, const int* sid,
                                        const int* s_nold, const int* s_pos, int* s_rslot, int* s_tslot,
                                        int* s_flag, int* s_rank, int* misc, uint32_t* bits, bool healthy,
@@ -744,9 +778,10 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
   size_t cell = 0;
   if (a.step.next.entry != nullptr && misc[13] >= 0) {
     const long long P2 = (long long)prefix[nst] + misc[13];
-    const long long Ge = P2 < G ? P2 : G;
-    c0 = blockIdx.x < Ge ? blockIdx.x * P2 / Ge : 0;
-    c1 = blockIdx.x < Ge ? (blockIdx.x + 1) * P2 / Ge : 0;
+    const Cut cut2(P2, nst, X, G);
+    auto pf2 = [&](int i) -> long long { return i < nst ? (long long)prefix[i] + s_rank[i] : P2; };
+    c0 = cut2.begin(blockIdx.x, nst, pf2);
+    c1 = cut2.begin(blockIdx.x + 1, nst, pf2);
     if (c1 - c0 <= a.step.next.cap) {
       cell = (size_t)wbuf * G + blockIdx.x;
       lst = a.step.next.list + cell * a.step.next.cap;
@@ -904,9 +939,8 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
         }
       }
       if (started) {
-        const long long P = prefix[nst];
-        const long long Geff = P < G ? P : G;
-        const int first = range_of(prefix[il], P, Geff), last = range_of(prefix[il + 1] - 1, P, Geff);
+        const Cut cut(prefix[nst], nst, X, G);
+        const int first = cut.owner(prefix[il], il), last = cut.owner(prefix[il + 1] - 1, il);
         const bool done = ld_acquire_gpu(&a.cnt[il]) == last - first;
         __threadfence_block();
         *reinterpret_cast<volatile int*>(&misc[3]) = done ? 1 : 2;
@@ -953,7 +987,8 @@ __host__ __device__ inline SmemLayout smem_layout(int ncw, int spw, int stage_by
 }
 
 // Split-K over CTA ranges. The call's retained pages, stream after stream,
-// are cut into gridDim.x equal contiguous ranges, one per CTA. Page c of a
+// are cut into gridDim.x contiguous ranges, one per CTA, of equal cost (pages,
+// plus a fixed cost for each stream piece: see Cut). Page c of a
 // range goes to warp c % NCW, which runs its own TMA pipeline over `spw`
 // private stages: it refills a stage as soon as it has computed on it, and
 // every stage's mbarrier phases are waited on by that one warp, in order.
@@ -968,16 +1003,17 @@ __host__ __device__ inline SmemLayout smem_layout(int ncw, int spw, int stage_by
 // it was before the step: the row of the token that leaves at this step is
 // masked, and the new token enters every stream's final merge from its input
 // row. A ninth warp resolves each stream's slots (window ring, page pops in
-// stream order, the same rule as dms_append) and, once every CTA has read
-// the pre-step state (grid-wide counter), writes the append: bookkeeping and
-// the K/V rows. A row it overwrites is a masked one or lies past the
-// pre-step count, so no CTA ever attends a row being written.
+// stream order, the same rule as dms_append) and writes the append:
+// bookkeeping into the other state parity and the K/V rows. A row it
+// overwrites is a masked one or lies past the pre-step count, so no CTA ever
+// attends a row being written, and no CTA waits for another.
 template <int D, int NCW, int NB, bool MMA, typename E, bool STEP>
 __global__ void __launch_bounds__((NCW + (STEP ? 1 : 0)) * 32, 1)
 attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   constexpr int kThreads = (NCW + (STEP ? 1 : 0)) * 32;   // consumers (+ the step warp)
   constexpr int kMergeThreads = NCW * 32;                  // the consumer warps
   constexpr int kStage = 2 * kPage * D * (int)sizeof(E);   // one page: 16 K rows + 16 V rows
+  constexpr int kX = piece_cost(D, MMA);                   // weight of a stream piece in the cut
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The 128-byte TMA swizzle needs 1024-aligned stages. The declaration asks
   // for that alignment and the launch reserves no slack for rounding up, so a
@@ -1000,7 +1036,8 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   // consumers' snapshot of [3]), [12] free-stack depth
   // and [13] pages popped by this step (-1: pool exhausted), [14] stream whose combine a split
   // first piece left to the end of the range (-1: none), [15] step decisions ready, [16] the
-  // status word the plan read, [17] STEP: the consumers have started the range's last piece
+  // status word the plan read, [17] STEP: the consumers have started the range's last piece,
+  // [18] and [19] the first and last CTA holding a piece of stream [14]
   int* misc = reinterpret_cast<int*>(smem + lay.misc);
   uint32_t* bits = reinterpret_cast<uint32_t*>(smem + lay.bits);
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(smem + lay.merge);
@@ -1083,7 +1120,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   // start of this launch with the end of the previous one.
   bool pre_ok = false;     // CTA-uniform: planned and copies issued before the wait
   bool any_miss = true;    // some stream of the call did not match the schedule
-  int pre_k0 = 0, pre_k1 = 0;   // this CTA's range in the guessed plan
+  int pre_k0 = 0, pre_k1 = 0;   // this CTA's range (in the guessed plan, then in the plan)
   using Query = typename std::conditional<MMA, MmaQuery<D>, SimtQuery<D>>::type;
   Query qcur;              // consumer lanes: the query of the piece about to start
   auto fetch_query = [&](int stream) {
@@ -1179,10 +1216,10 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
     bad |= gcount != a.n_seqs;
     pre_ok = !__syncthreads_or(bad) && misc[1] != 0;
     if (pre_ok) {
-      const long long P0 = prefix[nst];
-      const long long G0 = P0 < gridDim.x ? P0 : gridDim.x;
-      pre_k0 = blockIdx.x < G0 ? (int)(blockIdx.x * P0 / G0) : 0;
-      pre_k1 = blockIdx.x < G0 ? (int)((blockIdx.x + 1) * P0 / G0) : 0;
+      const Cut cut0(prefix[nst], nst, kX, gridDim.x);
+      auto pf = [&](int i) -> long long { return prefix[i]; };
+      pre_k0 = (int)cut0.begin(blockIdx.x, nst, pf);
+      pre_k1 = (int)cut0.begin(blockIdx.x + 1, nst, pf);
       if (warp < NCW) {
         const int nj = pre_k1 - pre_k0 > warp ? (pre_k1 - pre_k0 - warp + NCW - 1) / NCW : 0;
         if (lane < nj) {
@@ -1313,6 +1350,11 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       if (STEP) misc[12] = free_depth;
     }
     any_miss = __syncthreads_or(miss) != 0;
+    // This CTA's range (before any query fragment is held: the search needs registers).
+    const Cut cut(prefix[nst], nst, kX, gridDim.x);
+    auto pf = [&](int i) -> long long { return prefix[i]; };
+    pre_k0 = (int)cut.begin(blockIdx.x, nst, pf);
+    pre_k1 = (int)cut.begin(blockIdx.x + 1, nst, pf);
   }
   grid_dependents_launch();   // the next kernel may queue up behind this one
   if (STEP && tid == 0) misc[3] = 0;   // written by the step warp late in the launch
@@ -1324,9 +1366,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   if constexpr (!STEP) {
     if (!healthy) return;   // poisoned cache: do nothing (uniform over the CTA)
   }
-  const long long P = prefix[nst];
   const int G = gridDim.x;
-  const long long Geff = P < G ? P : G;
   if constexpr (!STEP) {
     // Streams with nothing retained produce zeros.
     for (int i = blockIdx.x; i < nst; i += G) {
@@ -1334,18 +1374,19 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
       const int b = i / a.hkv, kvh = i % a.hkv;
       for (int e = tid; e < a.g * D; e += kThreads) store_out(a, b, kvh * a.g + e / D, e % D, D, 0.f);
     }
-    if (blockIdx.x >= Geff) return;   // uniform over the CTA
   }
-  const bool has_range = healthy && blockIdx.x < Geff;
-  const int K0 = !has_range ? 0 : pre_ok ? pre_k0 : (int)(blockIdx.x * P / Geff);
-  const int K1 = !has_range ? 0 : pre_ok ? pre_k1 : (int)((blockIdx.x + 1) * P / Geff);
+  const int K0 = healthy ? pre_k0 : 0, K1 = healthy ? pre_k1 : 0;
+  const bool has_range = K1 > K0;
+  if constexpr (!STEP) {
+    if (!has_range) return;   // uniform over the CTA
+  }
   const int ncta = K1 - K0;
-  const bool list_ok = pre_ok || list_matches(P, ncta, any_miss);   // called once: it narrows thdr
+  const bool list_ok = pre_ok || list_matches(prefix[nst], ncta, any_miss);   // called once: it narrows thdr
   int consumed = 0, issued = 0;
   uint64_t* myfull = full + (warp < NCW ? warp : 0) * spw;
 
   if (STEP && warp == NCW) {
-    step_warp<D, E>(a, nst, prefix, sid, s_nold, s_pos, s_rslot, s_tslot, s_flag, s_rank, misc, bits, healthy,
+    step_warp<D, E, kX>(a, nst, prefix, sid, s_nold, s_pos, s_rslot, s_tslot, s_flag, s_rank, misc, bits, healthy,
                     abort_flag, K0, K1);
   } else if (STEP || has_range) {
     // ---- this warp's page pipeline: CTA pages c = warp + NCW * j, j = 0 .. njobs-1
@@ -1510,17 +1551,17 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
         // STEP, the range's last piece of a split stream: whether the step warp
         // has seen every other piece of it published (one snapshot for all).
         if (STEP && tid == 0 && !whole && pe == K1) misc[4] = *reinterpret_cast<volatile int*>(&misc[3]) == 1;
+        // Merge: thread t owns query head h = t / (D/4) and dims [4 d4, 4 d4 + 4);
+        // the CTA's result for its items stays in registers for the combine.
+        constexpr int kItems = kMaxGroup * D / 4;
+        constexpr int kIters = (kItems + kMergeThreads - 1) / kMergeThreads;
+        const int items = a.g * (D / 4);
         named_barrier(1, kMergeThreads);
         // (read from shared memory where it is used: a register held across the merge spills)
         auto known_last = [&]() -> bool {
           return STEP && !whole && pe == K1 && *reinterpret_cast<volatile int*>(&misc[4]) != 0;
         };
 
-        // Merge: thread t owns query head h = t / (D/4) and dims [4 d4, 4 d4 + 4);
-        // the CTA's result for its items stays in registers for the combine.
-        constexpr int kItems = kMaxGroup * D / 4;
-        constexpr int kIters = (kItems + kMergeThreads - 1) / kMergeThreads;
-        const int items = a.g * (D / 4);
         // The step warp's decisions are needed only by a merge that may finish
         // its stream (a whole piece, or the range's last piece, which may
         // combine); a split first piece only publishes its partial.
@@ -1574,12 +1615,17 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
           // Publish the partial: the CTA's stores, ordered by the barrier, are
           // released by thread 0's device-scope add; the adder that completes the
           // count acquires every other piece and combines.
-          const int first = range_of(pstart, P, Geff), last = range_of(pend - 1, P, Geff);
+          const Cut cut(prefix[nst], nst, kX, G);   // (from shared memory: nothing held across the pieces)
+          const int first = cut.owner(pstart, i), last = cut.owner(pend - 1, i);
           if (pe < K1) {
             // A split piece inside the range is its first piece. Thread 0
             // publishes it while the CTA goes on; a combine it finds due is done
             // by the whole CTA at the end of the range.
-            if (tid == 0 && atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first) misc[14] = i;
+            if (tid == 0 && atomic_add_acq_rel_gpu(&a.cnt[i], 1) == last - first) {
+              misc[14] = i;
+              misc[18] = first;
+              misc[19] = last;
+            }
           } else {
             const bool shortcut = known_last();
             if (shortcut) {
@@ -1635,8 +1681,7 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
   // ---- a split first piece that completed its stream: combine all its pieces
   __syncthreads();
   if (tid < kMergeThreads && misc[14] >= 0) {
-    const int i = misc[14];
-    const int first = range_of(prefix[i], P, Geff), last = range_of(prefix[i + 1] - 1, P, Geff);
+    const int i = misc[14], first = misc[18], last = misc[19];
     combine_stream<D, E, STEP>(a, i, first, last, tid, kMergeThreads, STEP && s_tslot[i] >= 0);
     if (tid == 0) a.cnt[i] = 0;   // ready for the next launch (stream order)
   }

@@ -16,6 +16,26 @@ constexpr int kMaxGroup = 8;       // query heads per KV head handled by one ker
 constexpr int kMaxStreams = 8192;  // max_seqs * num_kv_heads
 constexpr int kMaxKvHeads = 256;
 
+// What one stream piece costs a CTA of the tensor-core attention kernel, in
+// page-times, beyond its pages: the end-of-piece merge (a barrier that waits
+// for the warp holding the most pages of the piece, the merge of the warps'
+// states, the start of the next piece). The call's pages are cut into CTA
+// ranges with each stream weighted by it, so that a range that touches two
+// streams gets fewer pages than one inside a stream and both finish together.
+// The CUDA-core kernel, bound by arithmetic per page, is cut by pages alone, and
+// so is d = 64, whose short pieces measured no better with any weight.
+#ifndef DMS_PIECE_COST_D64
+#define DMS_PIECE_COST_D64 0
+#endif
+#ifndef DMS_PIECE_COST_D128
+#define DMS_PIECE_COST_D128 20
+#endif
+__host__ __device__ constexpr int piece_cost(int d, bool mma) {
+  return !mma ? 0 : d == 64 ? DMS_PIECE_COST_D64 : DMS_PIECE_COST_D128;
+}
+constexpr int kMaxPieceCost = DMS_PIECE_COST_D64 > DMS_PIECE_COST_D128 ? DMS_PIECE_COST_D64 : DMS_PIECE_COST_D128;
+static_assert(DMS_PIECE_COST_D64 >= 0 && DMS_PIECE_COST_D128 >= 0, "a piece cost is a page count");
+
 // Where the eviction decisions of appended tokens come from: an explicit
 // uint8 array [rows][hkv] (channel < 0), or the sign of one designated
 // channel of a projection row of each token (the eviction logit read from a
@@ -487,7 +507,7 @@ struct NextPlan {
   PlanEntry* entry;   // [2][S]
   int4* hdr;          // [2][grid][2]
   int32_t* list;      // [2][grid][cap]
-  int cap;            // page ids per CTA: enough for any range of any call (max_pages / grid, rounded up)
+  int cap;            // page ids per CTA: enough for any range of any call
   int S;              // entries per tag parity
 };
 // Where the eviction decisions of a fused step's new tokens come from: an
