@@ -665,9 +665,10 @@ def brief(res):
 
 
 def per_workload_runs(args, world, rank, local, dev, main_wl):
-    """The other workloads, each measured with fewer steps, no e2e and no CPU pass;
-    the long run at both ends of its decode loop; a dense (all kept) run of the
-    32K workload for context; the tiny workload as a correctness-only note."""
+    """The other workloads, each measured with fewer steps, no e2e and a short
+    oracle sample (all host cores and one core); the long run at both ends of its
+    decode loop; a dense (all kept) run of the 32K workload for context; the tiny
+    workload as a correctness-only note."""
     import dataclasses
     steps = min(args.steps, 20)
     runs = {}

@@ -630,7 +630,8 @@ __device__ __forceinline__ void step_warp(const AttnArgs& a, int nst, const int*
   const int par = a.par, nxt = par ^ 1;
   const Cur rd = cur_state(dv, par), wr = cur_state(dv, nxt);
   // Wait (no spinning) until the consumer warps have resolved every stream's
-  // leaving slot (s_rslot): they arrive at barrier 2 without waiting.
+  // leaving slot (s_rslot): they arrive at barrier 2 (waiting there too only
+  // when some slot came from the window ring).
   named_barrier(2, blockDim.x);
   if (healthy) {
     const int per = (nst + 31) / 32;   // contiguous streams per lane: the scan keeps stream order
@@ -1471,7 +1472,11 @@ attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmap) {
             s_rslot[il] = (s_pos[il] >= a.step.dv.w && (ring_v[q] & 1)) ? (ring_v[q] >> 1) : -1;
         }
       }
-      named_barrier_arrive(2, kThreads);   // hand them to the step warp (which syncs on barrier 2)
+      // Hand them to the step warp (which syncs on barrier 2). A consumer masks
+      // with the slots other consumer threads resolved, so when any was read from
+      // the ring here the consumers wait for all of them too (CTA-uniform).
+      if (!pre_ok && any_miss) named_barrier(2, kThreads);
+      else named_barrier_arrive(2, kThreads);
     }
     if (has_range) {
 

@@ -407,7 +407,10 @@ def test_fused_step_schedule_follows_every_change(case, caches):
                 out, Q = run.decode_step(step, seqs=arg, fused=kind == "fused")
                 torch.cuda.synchronize()
                 for j, b in enumerate(arg):
-                    compare(out[j], run.oracle_out(b, Q[j]), **tol)
+                    try:
+                        compare(out[j], run.oracle_out(b, Q[j]), **tol)
+                    except AssertionError as e:
+                        raise AssertionError(f"step {step} ({kind} {arg}), sequence {b}: {e}") from None
             for run in runs:
                 run.check_metadata()
         for run in runs:
