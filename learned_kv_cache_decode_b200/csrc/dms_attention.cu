@@ -962,9 +962,10 @@ __device__ __forceinline__ void issue_page(uint64_t* myfull, uint8_t* mystage, i
   mbar_arrive_expect_tx(bar, kStage);
   if constexpr (MMA) {
 #pragma unroll
-    for (int box = 0; box < D / 64; ++box) tma_load_3d(dst + box * 4096, tmap, bar, box * 64, 0, pg);
+    const uint64_t pol = l2_evict_first();   // pages are read once per launch
+    for (int box = 0; box < D / 64; ++box) tma_load_3d_hint(dst + box * 4096, tmap, bar, box * 64, 0, pg, pol);
   } else {
-    bulk_load(dst, kv + (size_t)pg * kStage, kStage, bar);
+    bulk_load_hint(dst, kv + (size_t)pg * kStage, kStage, bar, l2_evict_first());
   }
 }
 
