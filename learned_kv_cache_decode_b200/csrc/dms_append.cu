@@ -145,7 +145,7 @@ append_decode_kernel(Dev dv, int n_seqs, const int32_t* __restrict__ seq_ids,
       if (tid == 0) latch(dv.ctrl, DMS_ERR_POOL_EXHAUSTED);
       failed = 1;
     }
-    if (need && !fits) go = false;   // left unchanged: no stream of this round pops
+    if (need && !fits) go = false;   // left unchanged: no stream of this pass pops
     // ---- round trip 4
     int page = -1;
     if (go) {
